@@ -1,0 +1,101 @@
+"""The C-ABI library on the CPU: it builds, loads, exports every declared entry
+point, its host-only plan matches the oracle bit for bit, and host-side argument
+checks reject bad calls before anything touches a GPU."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import hsa_oracle as O
+from token_sparse_denoising_b200 import build, hsa
+from token_sparse_denoising_b200 import synthetic as S
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "hsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_library()
+    return hsa.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hsa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+@pytest.mark.parametrize("T,budgets,fracs,m,kind,shift,N", [
+    (8, [8, 4], (0.5, 0.5), 1, 0, 1.0, 1024),
+    (40, [40, 20, 10], (0.25, 0.25, 0.5), 4, 1, 5.0, 32760),
+    (40, [40, 8, 5, 1], (0.4, 0.2, 0.2, 0.2), 3, 1, 3.0, 1000),
+    (12, [12, 6, 4, 3], (0.25, 0.25, 0.25, 0.25), 0, 0, 1.0, 17),
+])
+def test_plan_matches_oracle_bit_exact(lib, T, budgets, fracs, m, kind, shift, N):
+    sizes = S.group_sizes(N, fracs)
+    sig, tab, nact = hsa.plan_groups(T, budgets, sizes, N, m, kind, shift)
+    assert sig.tobytes() == O.sigma_schedule(T, kind, shift).tobytes()
+    want_tab = O.active_table(T, budgets, m)
+    assert np.array_equal(tab.astype(bool), want_tab)
+    assert np.array_equal(nact, O.active_counts(want_tab, sizes))
+
+
+@pytest.mark.parametrize("bad", [dict(budgets=[8, 3]), dict(budgets=[4, 4]), dict(sizes=[4, 5]), dict(m=5),
+                                 dict(budgets=[4, 8]), dict(kind=2)])
+def test_plan_rejects(lib, bad):
+    a = dict(T=8, budgets=[8, 4], sizes=[4, 4], N=8, m=1, kind=0)
+    a.update(bad)
+    with pytest.raises(hsa.HsaError) as e:
+        hsa.plan_groups(a["T"], a["budgets"], a["sizes"], a["N"], a["m"], a["kind"], 1.0)
+    assert e.value.code == hsa.HSA_EINVAL
+
+
+def test_device_calls_reject_bad_arguments_on_host(lib):
+    null = None
+    sizes = (C.c_int * 2)(4, 4)
+    assert lib.hsa_select_tokens(null, 8, 0, sizes, null, null, null, 0, null) == hsa.HSA_EINVAL
+    assert lib.hsa_select_tokens(null, 8, 2, (C.c_int * 2)(4, 5), null, null, null, 0, null) == hsa.HSA_EINVAL
+    assert lib.hsa_euler_update(null, null, null, null, 0, 8, 6, 0.1, null, null) == hsa.HSA_EINVAL
+    assert lib.hsa_euler_update(null, null, null, null, 9, 8, 4, 0.1, null, null) == hsa.HSA_EINVAL
+    assert lib.hsa_l1_score(null, null, 4, 3, null, null) == hsa.HSA_EINVAL
+    assert lib.hsa_layer_step(null, null, null, 8, null, null, null, 1, null, null, null, 0, null, 0,
+                              null) == hsa.HSA_EINVAL
+    w = hsa.LayerWeightsC(300, 2, 64, hsa.HSA_BF16)           # D != 128 H
+    assert lib.hsa_layer_step(C.byref(w), null, null, 8, null, null, null, 1, null, null, null, 0, null, 0,
+                              null) == hsa.HSA_EINVAL
+    assert lib.hsa_linear(null, 4, 100, null, 64, null, hsa.HSA_BF16, 0, null, null, null) == hsa.HSA_EINVAL
+    assert lib.hsa_linear(null, 4, 64, null, 64, null, hsa.HSA_BF16, 9, null, null, null) == hsa.HSA_EINVAL
+    assert lib.hsa_linear(null, 0, 64, null, 64, null, hsa.HSA_BF16, 0, null, null, null) == hsa.HSA_OK
+    assert lib.hsa_attention(null, 0, null, null, 10, 1, hsa.HSA_BF16, null, null) == hsa.HSA_OK
+    assert lib.hsa_attention(null, 4, null, null, 10, 1, 7, null, null) == hsa.HSA_EINVAL
+    assert lib.hsa_context_kv(null, 0, 256, hsa.HSA_BF16, null, null, null, null, null, null, 0,
+                              null) == hsa.HSA_EINVAL
+    assert lib.hsa_patch_embed(null, null, 0, 8, 64, 256, hsa.HSA_BF16, null, null, null, null, 0,
+                               null) == hsa.HSA_EINVAL
+    assert b"need" in lib.hsa_last_error_string() or len(lib.hsa_last_error_string()) > 0
+
+
+def test_workspace_sizes(lib):
+    assert hsa.layer_step_workspace_size(32760, 1536, 8960, hsa.HSA_BF16) >= 32760 * (6 * 1536 + 8960) * 2
+    assert hsa.layer_step_workspace_size(1024, 256, 1024, hsa.HSA_F32) >= 1024 * (6 * 256 + 1024) * 4
+    assert lib.hsa_select_tokens_workspace_size(32760, 3) == 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    """No CPU fallback: a missing library is an error, not a silent substitute."""
+    saved = hsa._lib
+    try:
+        hsa._lib = None
+        with pytest.raises(RuntimeError):
+            hsa.load(str(tmp_path / "libhsa.so"))
+    finally:
+        hsa._lib = saved

@@ -1,0 +1,169 @@
+"""Parity of each CUDA building block with the oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import hsa_oracle as O
+from token_sparse_denoising_b200 import synthetic as S
+from tests._util import (assert_bf16_close, assert_f32_close, dev, host, max_abs, rel_l2)
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------------ §2.3 cached Euler + §2.1 score
+
+@pytest.mark.parametrize("N,C,M", [(1000, 64, 1000), (1000, 64, 377), (333, 1536, 333), (333, 1536, 100),
+                                   (7, 4, 0)])
+def test_euler_update(cuda_lib, N, C, M):
+    hsa = cuda_lib
+    x0, vh0 = S.normal(1, (N, C)), S.normal(2, (N, C))
+    vA = S.normal(3, (M, C))
+    idx = S.scattered_mask(4, N, M)
+    dsig = np.float32(-0.0375)
+    x, vh, va, ix = dev(x0), dev(vh0), dev(vA), dev(idx)
+    score = torch.full((N,), -1.0, device="cuda")
+    hsa.euler_update(x, vh, va if M else None, ix if M else None, float(dsig), score=score if M else None)
+    assert hsa.device_status() == 0
+    want_x, want_vh = O.cached_euler(x0, vh0, vA, idx, dsig)
+    assert_f32_close(host(x), want_x, "x")
+    assert np.array_equal(host(vh), want_vh.astype(np.float32))
+    if M:
+        want_s = O.l1_relative_change(vA, vh0[idx])
+        assert rel_l2(host(score)[idx], want_s) < 1e-5
+        untouched = np.setdiff1d(np.arange(N), idx)
+        assert np.all(host(score)[untouched] == -1.0)
+
+
+def test_l1_score(cuda_lib):
+    N, C = 5000, 1536
+    a, b = S.normal(5, (N, C)), S.normal(6, (N, C))
+    b[17] = 0.0                                          # zero previous velocity -> eps denominator
+    s = torch.empty(N, device="cuda")
+    cuda_lib.l1_score(dev(a), dev(b), s)
+    want = O.l1_relative_change(a, b)
+    got = host(s)
+    assert rel_l2(np.delete(got, 17), np.delete(want, 17)) < 1e-5
+    assert got[17] == pytest.approx(want[17], rel=1e-5)
+
+
+# ------------------------------------------------------------------ §2.1 selection: bit-exact
+
+def _select_case(seed, N, K, kind):
+    r = np.random.default_rng(seed)
+    if kind == "ties":
+        scores = r.choice(np.float32([0.0, 0.125, 0.5, 0.5000001, 1.0, np.nan, -1.0]), size=N).astype(np.float32)
+    elif kind == "const":
+        scores = np.full(N, 0.25, np.float32)
+    else:
+        scores = r.random(N, dtype=np.float32) * r.choice([1e-3, 1.0, 1e3], size=N).astype(np.float32)
+    cuts = np.sort(r.integers(0, N + 1, size=K - 1))
+    sizes = [int(v) for v in np.diff(np.concatenate([[0], cuts, [N]]))]
+    return scores, sizes
+
+
+@pytest.mark.parametrize("seed,N,K,kind", [(0, 1, 1, "rand"), (1, 5, 3, "ties"), (2, 1000, 2, "rand"),
+                                           (3, 1000, 4, "ties"), (4, 4097, 5, "const"), (5, 32760, 3, "rand"),
+                                           (6, 32760, 16, "ties"), (7, 75600, 3, "rand")])
+def test_select_tokens_bit_exact(cuda_lib, seed, N, K, kind):
+    scores, sizes = _select_case(seed, N, K, kind)
+    if seed == 5:
+        sizes = S.group_sizes(N, (0.25, 0.25, 0.5))
+    group = torch.full((N,), -7, dtype=torch.int8, device="cuda")
+    order = torch.full((N,), -7, dtype=torch.int32, device="cuda")
+    cuda_lib.select_tokens(dev(scores), sizes, group, order)
+    assert cuda_lib.device_status() == 0
+    want_g, want_o = O.select_groups(scores, sizes)
+    assert np.array_equal(host(group), want_g)
+    assert np.array_equal(host(order), want_o)
+
+
+# ------------------------------------------------------------------ linear layers
+
+def _lin_case(seed, M, K, Nout, bf16):
+    x = S.normal(seed, (M, K), 1.0, bf16)
+    w = S.normal(seed + 1, (Nout, K), 1.0 / np.sqrt(K), bf16)
+    b = S.normal(seed + 2, (Nout,), 0.1)
+    g = S.normal(seed + 3, (Nout,), 0.5)
+    y0 = S.normal(seed + 4, (M, Nout))
+    return x, w, b, g, y0
+
+
+@pytest.mark.parametrize("M,K,Nout", [(300, 256, 768), (129, 128, 64), (1000, 512, 384), (1, 64, 128),
+                                      (4097, 1536, 512)])
+@pytest.mark.parametrize("epi", [0, 1, 2, 3])
+def test_linear_bf16(cuda_lib, M, K, Nout, epi):
+    hsa = cuda_lib
+    x, w, b, g, y0 = _lin_case(11, M, K, Nout, True)
+    acc = O.linear(x, w, b)
+    if epi in (0, 1):
+        y = torch.empty((M, Nout), dtype=torch.bfloat16, device="cuda")
+        want = O.gelu_tanh(acc) if epi == 1 else acc
+    elif epi == 2:
+        y = dev(y0)
+        want = y0 + g * acc
+    else:
+        y = torch.empty((M, Nout), dtype=torch.float32, device="cuda")
+        want = acc
+    hsa.linear(dev(x, torch.bfloat16), dev(w, torch.bfloat16), dev(b), epi, y, gate=dev(g) if epi == 2 else None)
+    assert hsa.device_status() == 0
+    got = host(y)
+    if epi == 2:
+        assert_bf16_close(got - y0, want - y0, "residual delta")
+    else:
+        assert_bf16_close(got, want, f"epilogue {epi}")
+
+
+@pytest.mark.parametrize("M,K,Nout,epi", [(300, 256, 768, 0), (70, 128, 64, 1), (65, 256, 1024, 2)])
+def test_linear_f32(cuda_lib, M, K, Nout, epi):
+    x, w, b, g, y0 = _lin_case(21, M, K, Nout, False)
+    acc = O.linear(x, w, b)
+    y = dev(y0) if epi == 2 else torch.empty((M, Nout), device="cuda")
+    cuda_lib.linear(dev(x), dev(w), dev(b), epi, y, gate=dev(g) if epi == 2 else None)
+    want = {0: acc, 1: O.gelu_tanh(acc), 2: y0 + g * acc}[epi]
+    assert_f32_close(host(y), want)
+
+
+# ------------------------------------------------------------------ §2.2 attention
+
+@pytest.mark.parametrize("M,L,H,qscale", [(200, 1000, 2, 1.0), (128, 128, 1, 1.0), (1, 1, 1, 1.0),
+                                          (257, 300, 3, 4.0), (64, 4000, 2, 1.0)])
+def test_attention_bf16(cuda_lib, M, L, H, qscale):
+    D = 128 * H
+    q = S.normal(31, (M, D), qscale, True)
+    k, v = S.normal(32, (L, D), 1.0, True), S.normal(33, (L, D), 1.0, True)
+    o = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    cuda_lib.attention(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), H, o)
+    assert cuda_lib.device_status() == 0
+    assert_bf16_close(host(o), O.attention(q, k, v), "attention")
+
+
+def test_attention_rescale_across_tiles(cuda_lib):
+    """Logits that jump in a late key tile force the lazy O rescale."""
+    M, L, H = 130, 700, 1
+    q = S.normal(41, (M, 128), 1.0, True)
+    k = S.normal(42, (L, 128), 0.3, True)
+    v = S.normal(43, (L, 128), 1.0, True)
+    k[600:610] = S.round_bf16(np.repeat(q[:1] * 0.9, 10, 0))   # large logits for rows like q[0] late
+    k[300] = S.round_bf16(q[5] * 0.7)
+    o = torch.empty((M, 128), dtype=torch.bfloat16, device="cuda")
+    cuda_lib.attention(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), H, o)
+    assert_bf16_close(host(o), O.attention(q, k, v), "attention with late max")
+
+
+def test_attention_identical_keys_give_mean_value(cuda_lib):
+    M, L = 50, 513
+    q = S.normal(51, (M, 128), 1.0, True)
+    k = np.tile(S.normal(52, (1, 128), 1.0, True), (L, 1))
+    v = S.normal(53, (L, 128), 1.0, True)
+    o = torch.empty((M, 128), dtype=torch.bfloat16, device="cuda")
+    cuda_lib.attention(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), 1, o)
+    assert max_abs(host(o), np.tile(v.astype(np.float64).mean(0), (M, 1))) < 1e-2
+
+
+@pytest.mark.parametrize("M,L,H", [(100, 300, 2), (1, 1024, 1)])
+def test_attention_f32(cuda_lib, M, L, H):
+    D = 128 * H
+    q, k, v = S.normal(61, (M, D)), S.normal(62, (L, D)), S.normal(63, (L, D))
+    o = torch.empty((M, D), device="cuda")
+    cuda_lib.attention(dev(q), dev(k), dev(v), H, o)
+    assert_f32_close(host(o), O.attention(q, k, v))

@@ -1,0 +1,226 @@
+// gemm_tc.cu -- bf16 GEMM on the 5th-generation tensor cores for the linear
+// layers of the HSA block on the compacted active rows (HSA summary §2.2: only
+// A_i runs the projections and the feed-forward).
+//
+//   y[M x Nout] = epilogue(x[M x K] * W[Nout x K]^T + b)
+//
+// One CTA computes a 128 x BN tile.  Warp roles:
+//   warp 0      TMA producer: A (128 x 64) and B (BN x 64) k-blocks into a ring
+//               of STAGES shared-memory slots, 128-byte swizzled;
+//   warp 1      allocates BN TMEM columns; lane 0 issues tcgen05.mma
+//               (M=128, N=BN, K=16) into the fp32 TMEM accumulator and
+//               releases each slot with tcgen05.commit;
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter, bias, GELU /
+//               residual gate, 16-byte stores.  Thread = output row.
+// Rows beyond M are zero-filled by TMA and never stored.
+#include "tcgen05.cuh"
+
+namespace hsa {
+
+enum : int { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_F32 = 3 };
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 64;
+constexpr int kGemmThreads = 192;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kABytes = kGemmBM * kGemmBK * 2;   // 16 KB
+  static constexpr int kBBytes = BN * kGemmBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+__device__ __forceinline__ float gelu_tanh_f(float x) {
+  const float u = 0.7978845608028654f * (x + 0.044715f * x * x * x);
+  return 0.5f * x * (1.0f + tanhf(u));
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int Nout,
+              int K, const float* __restrict__ bias, const float* __restrict__ gate, void* __restrict__ out) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kGemmBM;
+  const int KB = K / kGemmBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t keep = policy_evict_last();   // weights are re-read by every row tile
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1)) break;
+        uint8_t* a = smem + s * Cfg::kStageBytes;
+        mbar_expect_tx(&full[s], Cfg::kStageBytes);
+        tma_load_2d(a, &tmA, &full[s], kb * kGemmBK, m0);
+        tma_load_2d_hint(a + Cfg::kABytes, &tmB, &full[s], kb * kGemmBK, n0, keep);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, BN, false);
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1;
+        if (!mbar_wait(&full[s], ph)) break;
+        tc_fence_after();
+        const uint32_t a = smem_u32(smem + s * Cfg::kStageBytes);
+        const uint32_t b = a + Cfg::kABytes;
+#pragma unroll
+        for (int k = 0; k < kGemmBK / 16; ++k) {
+          umma_ss(tmem, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), idesc,
+                  (kb | k) != 0);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(acc_full);
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows of that quarter
+    const int quarter = warp & 3;
+    const int row = m0 + quarter * 32 + lane;
+    mbar_wait(acc_full, 0);
+    __syncwarp();
+    tc_fence_after();
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the guarded stores
+      tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(c * 32), r);
+      tmem_ld_wait();
+      if (row < M) {
+        const int col0 = n0 + c * 32;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + (bias ? __ldg(bias + col0 + j) : 0.f);
+        if constexpr (EPI == EPI_STORE || EPI == EPI_GELU) {
+          __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * Nout + col0;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 u;
+            float t[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t[e] = EPI == EPI_GELU ? gelu_tanh_f(v[j + e]) : v[j + e];
+            u.x = pack_bf16x2(t[0], t[1]);
+            u.y = pack_bf16x2(t[2], t[3]);
+            u.z = pack_bf16x2(t[4], t[5]);
+            u.w = pack_bf16x2(t[6], t[7]);
+            *reinterpret_cast<uint4*>(y + j) = u;
+          }
+        } else if constexpr (EPI == EPI_F32) {
+          float* y = reinterpret_cast<float*>(out) + (size_t)row * Nout + col0;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(y + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        } else {  // EPI_RESID: y += gate * (acc + b)
+          float* y = reinterpret_cast<float*>(out) + (size_t)row * Nout + col0;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            float4 o = *reinterpret_cast<float4*>(y + j);
+            float g0 = 1.f, g1 = 1.f, g2 = 1.f, g3 = 1.f;
+            if (gate) {
+              g0 = __ldg(gate + col0 + j);
+              g1 = __ldg(gate + col0 + j + 1);
+              g2 = __ldg(gate + col0 + j + 2);
+              g3 = __ldg(gate + col0 + j + 3);
+            }
+            o.x = fmaf(g0, v[j], o.x);
+            o.y = fmaf(g1, v[j + 1], o.y);
+            o.z = fmaf(g2, v[j + 2], o.z);
+            o.w = fmaf(g3, v[j + 3], o.w);
+            *reinterpret_cast<float4*>(y + j) = o;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
+template <int BN, int EPI>
+static int launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, int M, int Nout, int K, const float* bias,
+                          const float* gate, void* out, cudaStream_t st) {
+  auto kern = k_gemm_tc<BN, EPI>;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::kSmem) != cudaSuccess)
+      return check_launch("gemm: shared-memory attribute");
+    attr_done[dev] = true;
+  }
+  dim3 grid(Nout / BN, (M + kGemmBM - 1) / kGemmBM);
+  kern<<<grid, kGemmThreads, GemmCfg<BN>::kSmem, st>>>(ta, tb, M, Nout, K, bias, gate, out);
+  count_launch(1);
+  return check_launch("gemm_tc launch");
+}
+
+template <int EPI>
+static int launch_gemm_epi(const void* A, int M, int K, const void* W, int Nout, const float* bias,
+                           const float* gate, void* out, cudaStream_t st) {
+  const int BN = (Nout % 256 == 0) ? 256 : (Nout % 128 == 0 ? 128 : 64);
+  CUtensorMap ta, tb;
+  int rc = make_tmap_2d(&ta, A, true, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, kGemmBK, kGemmBM, true);
+  if (rc) return rc;
+  rc = make_tmap_2d(&tb, W, true, (uint64_t)K, (uint64_t)Nout, (uint64_t)K * 2, kGemmBK, (uint32_t)BN, true);
+  if (rc) return rc;
+  if (BN == 256) return launch_gemm_bn<256, EPI>(ta, tb, M, Nout, K, bias, gate, out, st);
+  if (BN == 128) return launch_gemm_bn<128, EPI>(ta, tb, M, Nout, K, bias, gate, out, st);
+  return launch_gemm_bn<64, EPI>(ta, tb, M, Nout, K, bias, gate, out, st);
+}
+
+// Host entry used by every bf16 linear layer.  Shapes are validated here.
+int gemm_bf16(const void* A, int M, int K, const void* W, int Nout, const float* bias, int epi, const float* gate,
+              void* out, cudaStream_t st) {
+  if (M <= 0) return HSA_OK;
+  if (K <= 0 || K % kGemmBK || Nout <= 0 || Nout % 64)
+    return set_error(HSA_EINVAL, "bf16 linear: need K % 64 == 0 and Nout % 64 == 0");
+  if (!A || !W || !out || !aligned16(A) || !aligned16(W) || !aligned16(out))
+    return set_error(HSA_EINVAL, "bf16 linear: null or misaligned pointer");
+  switch (epi) {
+    case EPI_STORE: return launch_gemm_epi<EPI_STORE>(A, M, K, W, Nout, bias, gate, out, st);
+    case EPI_GELU: return launch_gemm_epi<EPI_GELU>(A, M, K, W, Nout, bias, gate, out, st);
+    case EPI_RESID: return launch_gemm_epi<EPI_RESID>(A, M, K, W, Nout, bias, gate, out, st);
+    case EPI_F32: return launch_gemm_epi<EPI_F32>(A, M, K, W, Nout, bias, gate, out, st);
+  }
+  return set_error(HSA_EINVAL, "linear: unknown epilogue");
+}
+
+}  // namespace hsa

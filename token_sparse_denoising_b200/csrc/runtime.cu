@@ -1,0 +1,102 @@
+// runtime.cu -- host side of libhsa: error text, the device status word, launch
+// counting and TMA tensor-map encoding.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "runtime.h"
+
+namespace hsa {
+
+static thread_local std::string t_last_error = "no error";
+static std::atomic<uint64_t> g_launches{0};
+
+int set_error(int code, const std::string& msg) {
+  t_last_error = msg;
+  return code;
+}
+
+int check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(HSA_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return HSA_OK;
+}
+
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int make_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+                 uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return set_error(HSA_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (!aligned16(base) || (row_stride_bytes & 15u))
+    return set_error(HSA_EINVAL, "tensor map base and row stride must be 16-byte aligned");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled failed (%d): dims %llu x %llu, box %u x %u", (int)r,
+             (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
+    return set_error(HSA_ECUDA, buf);
+  }
+  return HSA_OK;
+}
+
+}  // namespace hsa
+
+// ------------------------------------------------------------------ C ABI
+extern "C" const char* hsa_last_error_string(void) { return hsa::t_last_error.c_str(); }
+
+extern "C" uint64_t hsa_launch_count(void) { return hsa::g_launches.load(); }
+
+extern "C" int hsa_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(hsa::as_stream(stream));
+  if (e != cudaSuccess) return hsa::set_error(HSA_ECUDA, std::string("stream sync: ") + cudaGetErrorString(e));
+  int status = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&status, hsa::g_hsa_status, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(hsa::g_hsa_status, &zero, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(hsa::g_hsa_abort, &zero, sizeof(int));
+  if (e != cudaSuccess) return hsa::set_error(HSA_ECUDA, std::string("status word: ") + cudaGetErrorString(e));
+  if (status == HSA_EINDEX) hsa::set_error(status, "a kernel met a token index outside [0, N)");
+  if (status == HSA_ETIMEOUT) hsa::set_error(status, "a kernel's bounded pipeline wait ran out");
+  return status;
+}

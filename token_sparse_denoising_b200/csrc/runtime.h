@@ -1,0 +1,25 @@
+// runtime.h -- host-only declarations shared by the entry-point files of libhsa.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+namespace hsa {
+
+int set_error(int code, const std::string& msg);
+int check_launch(const char* what);
+void count_launch(int n);
+int num_sms();
+
+// 2-D tiled tensor map over a row-major matrix of `outer` rows x `inner` elements
+// (bf16 or f32), rows `row_stride_bytes` apart, boxes of box_outer x box_inner.
+int make_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+                 uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace hsa

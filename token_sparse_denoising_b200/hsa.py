@@ -1,0 +1,248 @@
+"""ctypes binding of libhsa.so (include/hsa.h): argument marshalling only.
+
+Every function takes torch tensors already on the device (or plain numbers)
+and passes their pointers, sizes and the current CUDA stream to the C ABI.
+There is no fallback: if libhsa.so cannot be loaded, `load()` raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libhsa.so")
+
+HSA_OK, HSA_EINVAL, HSA_EINDEX, HSA_ECUDA, HSA_ETIMEOUT, HSA_EWORKSPACE = range(6)
+HSA_F32, HSA_BF16 = 0, 1
+EPI_STORE, EPI_GELU, EPI_RESID, EPI_F32 = range(4)
+
+_lib = None
+vp, i32, u64, f32, sz = C.c_void_p, C.c_int, C.c_uint64, C.c_float, C.c_size_t
+
+
+class HsaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: status {code}: {_lib.hsa_last_error_string().decode()}")
+        self.code = code
+
+
+class LayerWeightsC(C.Structure):
+    _fields_ = [("D", i32), ("H", i32), ("F", i32), ("dtype", i32),
+                ("w_qkv", vp), ("b_qkv", vp), ("g_q", vp), ("g_k", vp),
+                ("w_o", vp), ("b_o", vp), ("w_1", vp), ("b_1", vp), ("w_2", vp), ("b_2", vp),
+                ("mod", vp), ("ln_c_g", vp), ("ln_c_b", vp), ("w_q2", vp), ("b_q2", vp), ("g_q2", vp),
+                ("w_o2", vp), ("b_o2", vp)]
+
+
+_SIGS = {
+    "hsa_last_error_string": (C.c_char_p, []),
+    "hsa_device_status": (i32, [vp]),
+    "hsa_launch_count": (u64, []),
+    "hsa_plan_groups": (i32, [i32, i32, vp, vp, i32, i32, i32, f32, vp, vp, vp]),
+    "hsa_l1_score": (i32, [vp, vp, i32, i32, vp, vp]),
+    "hsa_select_tokens_workspace_size": (sz, [i32, i32]),
+    "hsa_select_tokens": (i32, [vp, i32, i32, vp, vp, vp, vp, sz, vp]),
+    "hsa_euler_update": (i32, [vp, vp, vp, vp, i32, i32, i32, f32, vp, vp]),
+    "hsa_context_kv_workspace_size": (sz, [i32, i32]),
+    "hsa_context_kv": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
+    "hsa_layer_step_workspace_size": (sz, [i32, i32, i32, i32]),
+    "hsa_layer_step": (i32, [C.POINTER(LayerWeightsC), vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, i32, vp, sz, vp]),
+    "hsa_attention": (i32, [vp, i32, vp, vp, i32, i32, i32, vp, vp]),
+    "hsa_linear": (i32, [vp, i32, i32, vp, i32, vp, i32, i32, vp, vp, vp]),
+    "hsa_patch_workspace_size": (sz, [i32, i32, i32, i32]),
+    "hsa_patch_embed": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]),
+    "hsa_velocity_head": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
+}
+
+
+def load(path: str = LIB_PATH):
+    """Load libhsa.so (building it first when the in-tree copy is missing or stale)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path) or os.environ.get("HSA_REBUILD"):
+        from . import build
+        build.build_library()
+    if not os.path.exists(path):
+        raise RuntimeError(f"libhsa.so not found at {path}; the CUDA path has no fallback")
+    lib = C.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def lib():
+    return load()
+
+
+def _check(code: int, what: str):
+    if code != HSA_OK:
+        raise HsaError(code, what)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return HSA_BF16
+    if t.dtype == torch.float32:
+        return HSA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need(t, name, dtype=None):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+# ---------------------------------------------------------------- host plan
+
+def plan_groups(T: int, budgets, group_sizes, N: int, m: int, sigma_kind: int, shift: float):
+    """Returns (sigmas float32[T+1], active table uint8[T,K], n_active int32[T])."""
+    K = len(budgets)
+    b = np.ascontiguousarray(budgets, np.int32)
+    s = np.ascontiguousarray(group_sizes, np.int32)
+    sig = np.zeros(T + 1, np.float32)
+    tab = np.zeros((T, K), np.uint8)
+    nact = np.zeros(T, np.int32)
+    _check(lib().hsa_plan_groups(T, K, b.ctypes.data, s.ctypes.data, N, m, sigma_kind, shift,
+                                 sig.ctypes.data, tab.ctypes.data, nact.ctypes.data), "hsa_plan_groups")
+    return sig, tab, nact
+
+
+# ---------------------------------------------------------------- device calls
+
+def device_status(stream=None) -> int:
+    return lib().hsa_device_status(_stream(stream))
+
+
+def launch_count() -> int:
+    return int(lib().hsa_launch_count())
+
+
+def l1_score(v_new, v_prev, score, stream=None):
+    N, Cc = v_new.shape
+    _check(lib().hsa_l1_score(_ptr(v_new), _ptr(v_prev), N, Cc, _ptr(score), _stream(stream)), "hsa_l1_score")
+
+
+def select_tokens(score, group_sizes, group, order, stream=None):
+    import torch
+    N = score.shape[0]
+    K = len(group_sizes)
+    sizes = np.ascontiguousarray(group_sizes, np.int32)
+    nbytes = lib().hsa_select_tokens_workspace_size(N, K)
+    ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=score.device)
+    _check(lib().hsa_select_tokens(_ptr(score), N, K, sizes.ctypes.data, _ptr(group), _ptr(order), _ptr(ws),
+                                   nbytes, _stream(stream)), "hsa_select_tokens")
+
+
+def euler_update(x, vhat, vA, idx, dsigma: float, score=None, stream=None):
+    N, Cc = x.shape
+    M = 0 if idx is None else idx.shape[0]
+    _check(lib().hsa_euler_update(_ptr(x), _ptr(vhat), _ptr(vA), _ptr(idx), M, N, Cc, float(dsigma), _ptr(score),
+                                  _stream(stream)), "hsa_euler_update")
+
+
+def linear(x, w, b, epilogue: int, y, gate=None, stream=None):
+    M, K = x.shape
+    _check(lib().hsa_linear(_ptr(x), M, K, _ptr(w), w.shape[0], _ptr(b), _dtype_code(x), epilogue, _ptr(gate),
+                            _ptr(y), _stream(stream)), "hsa_linear")
+
+
+def attention(q, k, v, H: int, o, stream=None):
+    _check(lib().hsa_attention(_ptr(q), q.shape[0], _ptr(k), _ptr(v), k.shape[0], H, _dtype_code(q), _ptr(o),
+                               _stream(stream)), "hsa_attention")
+
+
+def context_kv_workspace_size(L: int, D: int) -> int:
+    return int(lib().hsa_context_kv_workspace_size(L, D))
+
+
+def context_kv(ctx, w_kv2, b_kv2, g_k2, k2, v2, ws, stream=None):
+    L, D = ctx.shape
+    _check(lib().hsa_context_kv(_ptr(ctx), L, D, _dtype_code(ctx), _ptr(w_kv2), _ptr(b_kv2), _ptr(g_k2), _ptr(k2),
+                                _ptr(v2), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "hsa_context_kv")
+
+
+def layer_step_workspace_size(M: int, D: int, F: int, dtype: int) -> int:
+    return int(lib().hsa_layer_step_workspace_size(M, D, F, dtype))
+
+
+def layer_step(w: "LayerWeights", kcache, vcache, xA, idx, pos, ws, x_src=None, ctx_k=None, ctx_v=None,
+               stream=None):
+    N = kcache.shape[0]
+    M = idx.shape[0]
+    L = 0 if ctx_k is None else ctx_k.shape[0]
+    _check(lib().hsa_layer_step(C.byref(w.c), _ptr(kcache), _ptr(vcache), N, _ptr(xA), _ptr(x_src), _ptr(idx), M,
+                                _ptr(pos), _ptr(ctx_k), _ptr(ctx_v), L, _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream(stream)), "hsa_layer_step")
+
+
+def patch_workspace_size(M: int, D: int, Cc: int, dtype: int) -> int:
+    return int(lib().hsa_patch_workspace_size(M, D, Cc, dtype))
+
+
+def patch_embed(x, idx, w_in, b_in, X, ws, stream=None):
+    N, Cc = x.shape
+    D = w_in.shape[0]
+    _check(lib().hsa_patch_embed(_ptr(x), _ptr(idx), idx.shape[0], N, Cc, D, _dtype_code(w_in), _ptr(w_in),
+                                 _ptr(b_in), _ptr(X), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "hsa_patch_embed")
+
+
+def velocity_head(X, head_mod, w_out, b_out, vA, ws, stream=None):
+    M, D = X.shape
+    _check(lib().hsa_velocity_head(_ptr(X), M, D, w_out.shape[0], _dtype_code(w_out), _ptr(head_mod), _ptr(w_out),
+                                   _ptr(b_out), _ptr(vA), _ptr(ws), ws.numel() * ws.element_size(),
+                                   _stream(stream)), "hsa_velocity_head")
+
+
+class LayerWeights:
+    """Device copies of one block's parameters plus the C struct that points at them."""
+
+    MATS = ("w_qkv", "w_o", "w_1", "w_2", "w_q2", "w_o2")
+    VECS = ("b_qkv", "g_q", "g_k", "b_o", "b_1", "b_2", "mod", "ln_c_g", "ln_c_b", "b_q2", "g_q2")
+
+    def __init__(self, bw, device, bf16: bool):
+        import torch
+        self.t = {}
+        mat_dtype = torch.bfloat16 if bf16 else torch.float32
+        for name in self.MATS:
+            a = getattr(bw, name)
+            if a is not None:
+                self.t[name] = torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device).to(mat_dtype)
+        for name in self.VECS:
+            a = getattr(bw, name)
+            if a is not None:
+                self.t[name] = torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
+        for name in ("w_kv2",):
+            if getattr(bw, name) is not None:
+                self.t[name] = torch.from_numpy(np.ascontiguousarray(bw.w_kv2, np.float32)).to(device).to(mat_dtype)
+                self.t["b_kv2"] = torch.from_numpy(np.ascontiguousarray(bw.b_kv2, np.float32)).to(device)
+                self.t["g_k2"] = torch.from_numpy(np.ascontiguousarray(bw.g_k2, np.float32)).to(device)
+        D, F = bw.w_o.shape[0], bw.w_1.shape[0]
+        self.D, self.H, self.F = D, D // 128, F
+        self.dtype = HSA_BF16 if bf16 else HSA_F32
+        p = lambda n: _ptr(self.t.get(n))
+        self.c = LayerWeightsC(D, D // 128, F, self.dtype, p("w_qkv"), p("b_qkv"), p("g_q"), p("g_k"), p("w_o"),
+                               p("b_o"), p("w_1"), p("b_1"), p("w_2"), p("b_2"), p("mod"), p("ln_c_g"),
+                               p("ln_c_b"), p("w_q2"), p("b_q2"), p("g_q2"), p("w_o2"), p("b_o2"))
