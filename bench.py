@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the HSA hot path at the Wan-1.3B block shape on B200.
+
+One step = one HSA denoising iteration of a Wan-1.3B-shaped DiT block (bf16,
+N = 32760 tokens from a 21x30x52 latent-patch grid, D = 1536, 12 heads, FFN
+8960, 512-token text context) with every token active, so every part of the
+hot path runs: gather + LayerNorm/modulation, QKV GEMM + q/k RMSNorm + 3D
+RoPE + KV-cache scatter, |A| x N attention, O-projection, cross-attention,
+FFN, velocity scatter + cached Euler with the fused L1 score, and the
+regrouping of the tokens (25/25/50 %).  A sweep times the layer step at
+|A|/N = 0.5 and 0.25 (active set: top-M tokens by L1 score of two velocity
+draws).  Inputs are seeded synthetic stand-ins (random-init weights).
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Multi-GPU: independent replicas, one per rank (the path has no exchange).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from token_sparse_denoising_b200 import synthetic as S  # noqa: E402
+
+METRIC = "HSA layer-step ms (Wan-1.3B block, |A|/N=1, full iteration)"
+GRID = S.WAN13_GRID
+SHAPE = S.WAN13_BLOCK
+GROUP_FRACS = (0.25, 0.25, 0.5)
+DSIGMA = -1.0 / 40.0
+SEED = 2
+ATTN_SRC = os.path.join(ROOT, "token_sparse_denoising_b200", "csrc", "attn_tc.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_traffic.json")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["hsa", "reference"], default="hsa")
+    p.add_argument("--no-sweep", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def workload_config(frac=1.0):
+    return {"workload": f"wan1.3b-block N={GRID.N} ({GRID.frames}x{GRID.height}x{GRID.width}) D={SHAPE.D} "
+                        f"H={SHAPE.H} F={SHAPE.F} ctx={SHAPE.ctx_len} |A|/N={frac:g}",
+            "tokens": GRID.N, "active_fraction": frac, "groups": list(GROUP_FRACS),
+            "l2": "no flush: the step's working set (~1.3 GB) is larger than the 126 MB L2",
+            "parallelism": "replicas"}
+
+
+def synthetic_inputs():
+    N, D = GRID.N, SHAPE.D
+    return {
+        "bw": S.block_weights(SEED, SHAPE, bf16=True),
+        "pos": S.token_positions(GRID),
+        "x0": S.normal(SEED * 10 + 1, (N, D)),
+        "vh0": S.normal(SEED * 10 + 2, (N, D)),
+        "ctx": S.normal(SEED * 10 + 3, (SHAPE.ctx_len, D), 1.0, True),
+        "kc0": S.normal(SEED * 10 + 4, (N, D), 1.0, True),
+        "vc0": S.normal(SEED * 10 + 5, (N, D), 1.0, True),
+        "va": S.normal(SEED * 10 + 6, (N, D)),
+        "vb": S.normal(SEED * 10 + 7, (N, D)),
+    }
+
+
+# ---------------------------------------------------------------- clocks during the timed region
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.path = tempfile.mktemp(suffix=".csv")
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- the CUDA path
+
+class Step:
+    """Device state of the workload and one HSA iteration through the C ABI."""
+
+    def __init__(self, inp, device):
+        import torch
+        from token_sparse_denoising_b200 import hsa, pipeline
+        self.torch, self.hsa = torch, hsa
+        N, D = GRID.N, SHAPE.D
+        self.N = N
+        self.sizes = S.group_sizes(N, GROUP_FRACS)
+        self.model = pipeline.SingleBlockModel(inp["bw"], inp["pos"], N, bf16=True, ctx=inp["ctx"],
+                                               cache_init=(inp["kc0"], inp["vc0"]), device=device)
+        self.x = torch.from_numpy(inp["x0"]).to(device)
+        self.vhat = torch.from_numpy(inp["vh0"]).to(device)
+        self.score = torch.zeros(N, device=device)
+        self.group = torch.zeros(N, dtype=torch.int8, device=device)
+        self.order = torch.arange(N, dtype=torch.int32, device=device)
+        # active sets of the sweep: top-M tokens by the L1 score of two velocity draws
+        va, vb = torch.from_numpy(inp["va"]).to(device), torch.from_numpy(inp["vb"]).to(device)
+        s = torch.empty(N, device=device)
+        hsa.l1_score(va, vb, s)
+        self.active = {}
+        for f in (0.5, 0.25):
+            M = S.active_fraction_rows(N, f)
+            g = torch.empty(N, dtype=torch.int8, device=device)
+            o = torch.empty(N, dtype=torch.int32, device=device)
+            hsa.select_tokens(s, [M, N - M], g, o)
+            self.active[f] = o[:M].clone()
+        del va, vb
+        torch.cuda.synchronize()
+
+    def full(self):
+        """One iteration with every token active (all rows of the hot path)."""
+        hsa = self.hsa
+        idx = self.order
+        vA = self.model.velocity(self.x, idx)
+        hsa.euler_update(self.x, self.vhat, vA, idx, DSIGMA, score=self.score)
+        hsa.select_tokens(self.score, self.sizes, self.group, self.order)
+
+    def partial(self, f):
+        """One iteration of the cached window: the layer step on the top-M set, then cached Euler."""
+        hsa = self.hsa
+        idx = self.active[f]
+        vA = self.model.velocity(self.x, idx)
+        hsa.euler_update(self.x, self.vhat, vA, idx, DSIGMA)
+
+
+def time_device(fn, steps, barrier):
+    import torch
+    st = torch.cuda.current_stream()
+    barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(steps):
+        fn()
+    b.record(st)
+    b.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    return a.elapsed_time(b)
+
+
+def attn_flops_per_full_step():
+    M = L = GRID.N
+    return 4.0 * M * L * 128 * SHAPE.H + 4.0 * M * SHAPE.ctx_len * 128 * SHAPE.H
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("bf16_tflops_sustained") or d["bf16_tflops"], d["bf16_tflops"], d["hbm_gbs"], "measured"
+    return 1400.0, 1590.0, 6650.0, "fallback"
+
+
+def traffic_per_launch():
+    """DRAM bytes of one attention launch from the committed ncu summary, if it is of this source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    sha = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
+    if d.get("source_sha256") != sha:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def run_gpu(args, rank, world, barrier, allmax):
+    import torch
+    from token_sparse_denoising_b200 import hsa
+    hsa.load()
+    device = torch.device("cuda", torch.cuda.current_device())
+    inp = synthetic_inputs()
+    step = Step(inp, device)
+    for _ in range(args.warmup):
+        step.full()
+    torch.cuda.synchronize()
+    assert hsa.device_status() == 0, "device status after warm-up"
+
+    # ---- timed region: K full iterations, per-kernel-class events on
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    hsa.timing_reset()
+    hsa.timing_enable(True)
+    l0 = hsa.launch_count()
+    ms = time_device(step.full, args.steps, barrier)
+    launches = hsa.launch_count() - l0
+    hsa.timing_enable(False)
+    attn_ms, attn_n = hsa.timing_read(hsa.KCLASS_ATTENTION)
+    gemm_ms, gemm_n = hsa.timing_read(hsa.KCLASS_GEMM)
+    other_ms, other_n = hsa.timing_read(hsa.KCLASS_OTHER)
+    hsa.timing_reset()
+    clk = clocks.stop() if clocks else None
+    ms_step = allmax(ms) / args.steps
+    status = hsa.device_status()
+    assert status == 0, f"device status {status}"
+
+    sweep = {}
+    if not args.no_sweep:
+        for f in (0.5, 0.25):
+            for _ in range(2):
+                step.partial(f)
+            sweep[str(f)] = allmax(time_device(lambda: step.partial(f), max(3, args.steps // 2), barrier)) / \
+                max(3, args.steps // 2)
+        sweep["1.0"] = ms_step
+
+    e2e = None
+    if not args.no_e2e:
+        # end to end through the public API with host buffers: the latent goes host -> device
+        # before each iteration and comes back after it (pinned memory, copies timed)
+        hx = torch.from_numpy(inp["x0"]).pin_memory()
+        hout = torch.empty_like(hx).pin_memory()
+
+        def e2e_step():
+            step.x.copy_(hx, non_blocking=True)
+            step.full()
+            hout.copy_(step.x, non_blocking=True)
+        e2e_step()
+        n_e2e = max(3, args.steps // 2)
+        e_ms = allmax(time_device(e2e_step, n_e2e, barrier)) / n_e2e
+        nbytes = GRID.N * SHAPE.D * 4
+        e2e = {"value": round(e_ms, 4), "unit": "ms", "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+
+    peak_sus, peak_burst, hbm, src = load_peaks()
+    attn_per_step = attn_ms / args.steps
+    achieved = attn_flops_per_full_step() / (attn_per_step * 1e-3) / 1e12
+    traffic = traffic_per_launch()
+    out = {
+        "metric": METRIC, "value": round(ms_step, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded random-init weights and inputs)",
+        "config": workload_config(1.0),
+        "roofline": {"bound": "tensor", "kernel": "k_attn_tc (self + cross attention launches)",
+                     "achieved": round(achieved, 1), "peak": peak_sus, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_sus, 4),
+                     "peak_note": f"{src} sustained bf16 (burst {peak_burst}: frac {achieved / peak_burst:.3f})",
+                     "traffic": traffic, "launches_per_step": attn_n // max(args.steps, 1),
+                     "flops_per_step": attn_flops_per_full_step()},
+        "breakdown_ms_per_step": {"attention": round(attn_per_step, 4), "gemm": round(gemm_ms / args.steps, 4),
+                                  "other": round(other_ms / args.steps, 4)},
+        "sweep_ms": {k: round(v, 4) for k, v in sweep.items()},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    return out
+
+
+# ---------------------------------------------------------------- the oracle on the host cores
+
+ORACLE_ROWS = 32        # attention / O / cross / FFN query rows per sample
+ORACLE_PROJ = 4096      # tokens whose q/k/v projections, Euler update and score run per sample
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_step_sample(inp):
+    """Time the oracle on a bounded sample of one full iteration; return the extrapolated ms per step.
+
+    Every part of the step is linear in the rows it touches, so each is timed on
+    a spread sample and scaled: the q/k/v projections (LN, GEMM, RMSNorm, RoPE)
+    and the cached Euler update + L1 score of ORACLE_PROJ tokens (x N/4096);
+    attention over all N cache rows + O-projection + cross-attention + FFN of
+    ORACLE_ROWS query rows (x N/32); the regrouping runs on all N scores.
+    """
+    from oracle import hsa_oracle as O
+    N = GRID.N
+    bw, pos = inp["bw"], inp["pos"]
+    ctx_kv = O.context_kv(bw, inp["ctx"])            # once per run: not part of a step
+    proj = np.arange(0, N, N // ORACLE_PROJ)[:ORACLE_PROJ]
+    qrows = np.arange(0, ORACLE_PROJ, ORACLE_PROJ // ORACLE_ROWS)[:ORACLE_ROWS]
+    X = inp["x0"][proj].astype(np.float64)
+    Kc, Vc = inp["kc0"].astype(np.float64), inp["vc0"].astype(np.float64)
+    t0 = time.perf_counter()
+    q, k, v = O.qkv_projection(bw, X, pos[proj])
+    Kc[proj], Vc[proj] = k, v
+    t1 = time.perf_counter()
+    O.block_tail(bw, X[qrows], O.attention(q[qrows], Kc, Vc), ctx_kv)
+    t2 = time.perf_counter()
+    vA = inp["va"][proj].astype(np.float64)          # a stand-in velocity of the same shape
+    score = O.l1_relative_change(vA, inp["vh0"][proj])
+    O.cached_euler(inp["x0"][proj], inp["vh0"][proj], vA, np.arange(len(proj)), DSIGMA)
+    t3 = time.perf_counter()
+    O.select_groups(np.resize(score.astype(np.float32), N), S.group_sizes(N, GROUP_FRACS))
+    t4 = time.perf_counter()
+    per_token = (t1 - t0) + (t3 - t2)
+    est_ms = (per_token * N / len(proj) + (t2 - t1) * N / len(qrows) + (t4 - t3)) * 1e3
+    sample = (f"fp64 numpy oracle; q/k/v projections + Euler/score of {len(proj)} of {N} tokens "
+              f"({per_token:.2f} s, x{N / len(proj):.1f}), attention over all {N} cache rows + O/cross/FFN of "
+              f"{len(qrows)} query rows ({t2 - t1:.2f} s, x{N / len(qrows):.0f}), regrouping of {N} scores "
+              f"({t4 - t3:.2f} s)")
+    return est_ms, (t4 - t0), sample
+
+
+def cpu_baseline(inp):
+    est_ms, wall, sample = oracle_step_sample(inp)
+    return {"value": round(est_ms, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
+            "sample": sample, "wall_s": round(wall, 2)}
+
+
+def run_reference(args):
+    inp = synthetic_inputs()
+    for _ in range(args.warmup):
+        oracle_step_sample(inp)
+    vals, wall, sample = [], 0.0, ""
+    for _ in range(args.steps):
+        v, w, sample = oracle_step_sample(inp)
+        vals.append(v)
+        wall += w
+    value = float(np.mean(vals))
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "ms", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value, 1), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(1.0),
+            "cpu_baseline": {"value": round(value, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": round(wall, 1)}
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def allmax(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    try:
+        out = run_gpu(args, rank, world, barrier, allmax)
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(synthetic_inputs())
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -66,6 +66,16 @@ int hsa_device_status(void* stream);
 /* Number of kernel launches the library has enqueued in this process. */
 uint64_t hsa_launch_count(void);
 
+/* Per-kernel timing (measurement support; off by default).  While enabled, every
+ * launch libhsa makes is bracketed by two CUDA events recorded on its stream,
+ * filed under a kernel class.  hsa_timing_read waits for the recorded events
+ * and returns the summed device time (ms) and the launch count of one class;
+ * hsa_timing_reset forgets every record.  Host state of this process. */
+enum { HSA_KCLASS_ATTENTION = 0, HSA_KCLASS_GEMM = 1, HSA_KCLASS_OTHER = 2, HSA_KCLASS_COUNT = 3 };
+int hsa_timing_enable(int on);
+int hsa_timing_read(int kclass, double* total_ms, int* launches);
+int hsa_timing_reset(void);
+
 /* ------------------------------------------------------------------ §2.1 + §2.4 plan (host only)
  * Validates (T, K, s_k, n_k, N, m) and writes the schedule of the whole run.
  *   h_budgets[K]      s_k; s_1 = T, every s_k divides T, non-increasing.

@@ -98,10 +98,69 @@ def test_tiny_fp32_loop_matches_oracle(cuda_lib):
 
     zeros = np.zeros((N, D))
     final, states = O.hsa_denoise(x0, vh0, plan, vel, (zeros, zeros), keep_states=True)
+    swapped = set()
     for r, st in zip(rec, states):
         assert r["M"] == len(st["idx"])
         if r["full"]:
             assert rel_l2(r["score"], st["score"]) < 1e-4
-            assert np.array_equal(r["order"], st["order"])
-    assert_f32_close(x_gpu, final["x"], "final latent")
-    assert_f32_close(x_gpu - x0, final["x"] - x0, "latent displacement")
+            swapped |= _near_tie_swaps(r["order"], st["order"], st["score"], sizes)
+    # tokens on a near-tied group boundary may run a step later on one side; they
+    # must be few, and every other token must match
+    assert len(swapped) <= 8, f"{len(swapped)} tokens changed group"
+    keep = np.setdiff1d(np.arange(N), np.array(sorted(swapped), dtype=np.int64))
+    assert_f32_close(x_gpu[keep], final["x"][keep], "final latent")
+    assert_f32_close(x_gpu[keep] - x0[keep], final["x"][keep] - x0[keep], "latent displacement")
+
+
+def _near_tie_swaps(order_gpu, order_ref, score_ref, sizes, rel=1e-5):
+    """Tokens whose group differs between the two partitions; each must sit on a near-tied boundary."""
+    starts = np.concatenate([[0], np.cumsum(sizes)])
+    g_gpu = np.empty(len(order_gpu), np.int64)
+    g_ref = np.empty(len(order_ref), np.int64)
+    for k in range(len(sizes)):
+        g_gpu[order_gpu[starts[k]:starts[k + 1]]] = k
+        g_ref[order_ref[starts[k]:starts[k + 1]]] = k
+    diff = np.nonzero(g_gpu != g_ref)[0]
+    srt = np.sort(score_ref)[::-1]
+    for n in diff:
+        k = min(g_gpu[n], g_ref[n])
+        boundary = srt[starts[k + 1] - 1]                      # lowest score kept in the higher group
+        assert abs(score_ref[n] - boundary) <= rel * abs(boundary), \
+            f"token {n} changed group with score {score_ref[n]} far from the boundary {boundary}"
+    return set(int(n) for n in diff)
+
+
+def test_wan_loop_standin_bf16_matches_oracle(cuda_lib):
+    """Reduced stand-in of the Wan-1.3B loop: patch model (C=64) with 3 bf16 blocks with cross-attention,
+    T=40, budgets {40,20,10} sized 25/25/50 %, m=4, shifted sigma (shift 5), N = 1x8x16 tokens."""
+    wl = S.WAN13_LOOP_SMALL
+    N, C = wl.grid.N, wl.C
+    pm = S.patch_model_weights(wl.seed, wl.shape, C, wl.n_blocks, True, std=0.05)
+    pos = S.token_positions(wl.grid)
+    x0, vh0 = S.normal(wl.seed * 10 + 1, (N, C)), S.normal(wl.seed * 10 + 2, (N, C))
+    ctx = S.normal(wl.seed * 10 + 3, (wl.shape.ctx_len, wl.shape.D), 1.0, True)
+    sizes = S.group_sizes(N, wl.fracs)
+    model = pipeline.PatchModel(pm, pos, N, bf16=True, ctx=ctx)
+    run = pipeline.HSARun(model, x0, vh0, wl.T, wl.budgets, sizes, wl.m, wl.sigma_kind, wl.shift)
+    rec = []
+    x_gpu = host(run.run(rec))
+    assert hsa.device_status() == 0
+
+    plan = O.make_plan(wl.T, wl.budgets, sizes, wl.m, wl.sigma_kind, wl.shift, N)
+    ctx_kvs = [O.context_kv(bw, ctx) for bw in pm.blocks]
+
+    def vel(xA, idx, caches):
+        v, new = O.patch_model_active(pm, xA, idx, pos, caches, ctx_kvs)
+        return v, new
+
+    zeros = [(np.zeros((N, wl.shape.D)), np.zeros((N, wl.shape.D))) for _ in pm.blocks]
+    final, states = O.hsa_denoise(x0, vh0, plan, vel, zeros, keep_states=True)
+    swapped = set()
+    for r, st in zip(rec, states):
+        assert r["M"] == len(st["idx"])
+        if r["full"]:
+            assert rel_l2(r["score"], st["score"]) < 2e-2
+            swapped |= _near_tie_swaps(r["order"], st["order"], st["score"], sizes, rel=3e-2)
+    assert len(swapped) <= N // 8, f"{len(swapped)} tokens changed group"
+    keep = np.setdiff1d(np.arange(N), np.array(sorted(swapped), dtype=np.int64))
+    assert_bf16_close(x_gpu[keep] - x0[keep], final["x"][keep] - x0[keep], "latent displacement")

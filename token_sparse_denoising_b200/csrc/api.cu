@@ -27,6 +27,7 @@ static inline size_t esize(int dtype) { return dtype == HSA_BF16 ? 2 : 4; }
 template <typename TOut>
 static int launch_ln(float* X, const float* x_src, const int* idx, int M, int N, int D, const float* mul,
                      const float* add, int plus_one, TOut* h, cudaStream_t st) {
+  ScopedTiming timing(HSA_KCLASS_OTHER, st);
   const unsigned g = warp_blocks(M);
   switch (D / 128 * (D % 128 == 0)) {
     case 1: k_ln_rows<1, TOut><<<g, 256, 0, st>>>(X, x_src, idx, M, N, mul, add, plus_one, h); break;
@@ -44,6 +45,7 @@ static int launch_ln(float* X, const float* x_src, const int* idx, int M, int N,
 template <typename T>
 static int launch_qk_rope(const T* qkv, const int* idx, const int* pos, int M, int N, int D, const float* g_q,
                           const float* g_k, T* Q, T* Kc, T* Vc, cudaStream_t st) {
+  ScopedTiming timing(HSA_KCLASS_OTHER, st);
   const unsigned g = warp_blocks(M);
   switch (D / 128) {
     case 1: k_qk_norm_rope<1, T, T><<<g, 256, 0, st>>>(qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
@@ -60,6 +62,7 @@ static int launch_qk_rope(const T* qkv, const int* idx, const int* pos, int M, i
 template <typename T>
 static int launch_rms(const T* in, int in_stride, int M, int D, const float* g, T* out, cudaStream_t st) {
   if (M <= 0) return HSA_OK;
+  ScopedTiming timing(HSA_KCLASS_OTHER, st);
   k_rms_rows<T, T><<<warp_blocks(M), 256, 0, st>>>(in, in_stride, M, D, g, out);
   count_launch(1);
   return check_launch("rms rows launch");
@@ -91,6 +94,7 @@ extern "C" int hsa_l1_score(const float* d_v_new, const float* d_v_prev, int N, 
   if (N == 0) return HSA_OK;
   if (!d_v_new || !d_v_prev || !d_score || !aligned16(d_v_new) || !aligned16(d_v_prev))
     return set_error(HSA_EINVAL, "l1_score: null or misaligned pointer");
+  ScopedTiming timing(HSA_KCLASS_OTHER, as_stream(stream));
   k_l1_score<<<warp_blocks(N), 256, 0, as_stream(stream)>>>(d_v_new, d_v_prev, N, C, d_score);
   count_launch(1);
   return check_launch("l1_score launch");
@@ -104,6 +108,7 @@ extern "C" int hsa_euler_update(float* d_x, float* d_vhat, const float* d_vA, co
     return set_error(HSA_EINVAL, "euler: null or misaligned x / v_hat");
   if (M > 0 && (!d_vA || !d_idx || !aligned16(d_vA))) return set_error(HSA_EINVAL, "euler: null v_A or idx");
   cudaStream_t st = as_stream(stream);
+  ScopedTiming timing(HSA_KCLASS_OTHER, st);
   if (M == N) {
     // every token active: scatter, score and Euler in one pass over the rows
     k_scatter_vhat<<<warp_blocks(M), 256, 0, st>>>(d_vhat, d_vA, d_idx, M, N, C, d_score, d_x, dsigma);
@@ -271,6 +276,7 @@ extern "C" int hsa_patch_embed(const float* d_x, const int32_t* d_idx, int M, in
     return set_error(HSA_EINVAL, "patch_embed: null or misaligned pointer");
   if (ws_bytes < hsa_patch_workspace_size(M, D, C, dtype)) return set_error(HSA_EWORKSPACE, "patch_embed: workspace");
   cudaStream_t st = as_stream(stream);
+  ScopedTiming timing(HSA_KCLASS_OTHER, st);
   if (dtype == HSA_BF16)
     k_gather_rows<__nv_bfloat16><<<warp_blocks(M), 256, 0, st>>>(d_x, d_idx, M, N, C, static_cast<__nv_bfloat16*>(d_ws));
   else

@@ -275,6 +275,7 @@ int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, in
     attr_done[dev] = true;
   }
   dim3 grid((M + kAttnBM - 1) / kAttnBM, H);
+  ScopedTiming timing(HSA_KCLASS_ATTENTION, st);
   k_attn_tc<<<grid, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, M, L, H, reinterpret_cast<__nv_bfloat16*>(O));
   count_launch(1);
   return check_launch("attn_tc launch");

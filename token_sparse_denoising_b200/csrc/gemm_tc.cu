@@ -187,6 +187,7 @@ static int launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, int M, i
     attr_done[dev] = true;
   }
   dim3 grid(Nout / BN, (M + kGemmBM - 1) / kGemmBM);
+  ScopedTiming timing(HSA_KCLASS_GEMM, st);
   kern<<<grid, kGemmThreads, GemmCfg<BN>::kSmem, st>>>(ta, tb, M, Nout, K, bias, gate, out);
   count_launch(1);
   return check_launch("gemm_tc launch");

@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "common.cuh"
 #include "runtime.h"
@@ -81,9 +82,86 @@ int make_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, 
   return HSA_OK;
 }
 
+// ------------------------------------------------------------------ per-kernel timing
+namespace {
+struct TimingRec {
+  cudaEvent_t a, b;
+  int kclass;
+};
+std::mutex g_tmu;
+bool g_timing = false;
+std::vector<TimingRec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+}  // namespace
+
+ScopedTiming::ScopedTiming(int kclass, cudaStream_t st) : kclass_(kclass), st_(st) {
+  std::lock_guard<std::mutex> g(g_tmu);
+  if (!g_timing) return;
+  a_ = take_event();
+  if (a_) cudaEventRecord(a_, st_);
+}
+
+ScopedTiming::~ScopedTiming() {
+  if (!a_) return;
+  std::lock_guard<std::mutex> g(g_tmu);
+  cudaEvent_t b = take_event();
+  if (!b) {
+    g_pool.push_back(a_);
+    return;
+  }
+  cudaEventRecord(b, st_);
+  g_recs.push_back({a_, b, kclass_});
+}
+
 }  // namespace hsa
 
 // ------------------------------------------------------------------ C ABI
+extern "C" int hsa_timing_enable(int on) {
+  std::lock_guard<std::mutex> g(hsa::g_tmu);
+  hsa::g_timing = on != 0;
+  return HSA_OK;
+}
+
+extern "C" int hsa_timing_read(int kclass, double* total_ms, int* launches) {
+  if (kclass < 0 || kclass >= HSA_KCLASS_COUNT || !total_ms || !launches)
+    return hsa::set_error(HSA_EINVAL, "timing_read: bad class or null output");
+  std::lock_guard<std::mutex> g(hsa::g_tmu);
+  double ms = 0.0;
+  int n = 0;
+  for (const auto& r : hsa::g_recs) {
+    if (r.kclass != kclass) continue;
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return hsa::check_launch("timing_read: event sync");
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) return hsa::check_launch("timing_read: elapsed");
+    ms += t;
+    ++n;
+  }
+  *total_ms = ms;
+  *launches = n;
+  return HSA_OK;
+}
+
+extern "C" int hsa_timing_reset(void) {
+  std::lock_guard<std::mutex> g(hsa::g_tmu);
+  for (auto& r : hsa::g_recs) {
+    cudaEventSynchronize(r.b);
+    hsa::g_pool.push_back(r.a);
+    hsa::g_pool.push_back(r.b);
+  }
+  hsa::g_recs.clear();
+  return HSA_OK;
+}
 extern "C" const char* hsa_last_error_string(void) { return hsa::t_last_error.c_str(); }
 
 extern "C" uint64_t hsa_launch_count(void) { return hsa::g_launches.load(); }

@@ -19,6 +19,21 @@ int num_sms();
 int make_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
 
+// Records a CUDA event pair around the launches made while it is alive, when
+// timing is enabled (hsa_timing_enable); otherwise does nothing.
+class ScopedTiming {
+ public:
+  ScopedTiming(int kclass, cudaStream_t st);
+  ~ScopedTiming();
+  ScopedTiming(const ScopedTiming&) = delete;
+  ScopedTiming& operator=(const ScopedTiming&) = delete;
+
+ private:
+  int kclass_;
+  cudaStream_t st_;
+  cudaEvent_t a_ = nullptr;
+};
+
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

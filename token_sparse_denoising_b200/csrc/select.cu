@@ -188,6 +188,7 @@ extern "C" int hsa_select_tokens(const float* d_score, int N, int K, const int* 
   }
   if (c != N) return set_error(HSA_EINVAL, "select: group sizes must sum to N");
   if (N == 0) return HSA_OK;
+  ScopedTiming timing(HSA_KCLASS_OTHER, as_stream(stream));
   k_select<<<1, kSelectThreads, 0, as_stream(stream)>>>(d_score, N, a, d_group, d_order);
   count_launch(1);
   return check_launch("select launch");

@@ -70,6 +70,7 @@ int gemm_f32(const float* A, int M, int K, const float* W, int Nout, const float
   if (!A || !W || !out || !aligned16(A) || !aligned16(W) || !aligned16(out))
     return set_error(HSA_EINVAL, "f32 linear: null or misaligned pointer");
   dim3 grid((Nout + 63) / 64, (M + 63) / 64);
+  ScopedTiming timing(HSA_KCLASS_GEMM, st);
   switch (epi) {
     case 1: k_gemm_f32<1><<<grid, 256, 0, st>>>(A, W, M, Nout, K, bias, gate, out); break;
     case 2: k_gemm_f32<2><<<grid, 256, 0, st>>>(A, W, M, Nout, K, bias, gate, out); break;
@@ -118,6 +119,7 @@ int attention_f32(const float* Q, int M, const float* K, const float* V, int L, 
   if (M <= 0) return HSA_OK;
   if (L <= 0 || H <= 0) return set_error(HSA_EINVAL, "attention: need L > 0 and H > 0");
   const long long warps = (long long)M * H;
+  ScopedTiming timing(HSA_KCLASS_ATTENTION, st);
   k_attn_f32<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(Q, M, K, V, L, H, O);
   count_launch(1);
   return check_launch("attn_f32 launch");

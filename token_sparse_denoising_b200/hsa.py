@@ -40,6 +40,9 @@ _SIGS = {
     "hsa_last_error_string": (C.c_char_p, []),
     "hsa_device_status": (i32, [vp]),
     "hsa_launch_count": (u64, []),
+    "hsa_timing_enable": (i32, [i32]),
+    "hsa_timing_read": (i32, [i32, C.POINTER(C.c_double), C.POINTER(i32)]),
+    "hsa_timing_reset": (i32, []),
     "hsa_plan_groups": (i32, [i32, i32, vp, vp, i32, i32, i32, f32, vp, vp, vp]),
     "hsa_l1_score": (i32, [vp, vp, i32, i32, vp, vp]),
     "hsa_select_tokens_workspace_size": (sz, [i32, i32]),
@@ -138,6 +141,24 @@ def launch_count() -> int:
     return int(lib().hsa_launch_count())
 
 
+KCLASS_ATTENTION, KCLASS_GEMM, KCLASS_OTHER = 0, 1, 2
+
+
+def timing_enable(on: bool = True):
+    _check(lib().hsa_timing_enable(1 if on else 0), "hsa_timing_enable")
+
+
+def timing_read(kclass: int):
+    """(summed device ms, launch count) of one kernel class since the last reset."""
+    ms, n = C.c_double(0.0), i32(0)
+    _check(lib().hsa_timing_read(kclass, C.byref(ms), C.byref(n)), "hsa_timing_read")
+    return ms.value, n.value
+
+
+def timing_reset():
+    _check(lib().hsa_timing_reset(), "hsa_timing_reset")
+
+
 def l1_score(v_new, v_prev, score, stream=None):
     N, Cc = v_new.shape
     _check(lib().hsa_l1_score(_ptr(v_new), _ptr(v_prev), N, Cc, _ptr(score), _stream(stream)), "hsa_l1_score")
@@ -220,7 +241,7 @@ class LayerWeights:
     """Device copies of one block's parameters plus the C struct that points at them."""
 
     MATS = ("w_qkv", "w_o", "w_1", "w_2", "w_q2", "w_o2")
-    VECS = ("b_qkv", "g_q", "g_k", "b_o", "b_1", "b_2", "mod", "ln_c_g", "ln_c_b", "b_q2", "g_q2")
+    VECS = ("b_qkv", "g_q", "g_k", "b_o", "b_1", "b_2", "mod", "ln_c_g", "ln_c_b", "b_q2", "g_q2", "b_o2")
 
     def __init__(self, bw, device, bf16: bool):
         import torch
