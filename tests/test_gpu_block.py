@@ -155,12 +155,20 @@ def test_wan_loop_standin_bf16_matches_oracle(cuda_lib):
 
     zeros = [(np.zeros((N, wl.shape.D)), np.zeros((N, wl.shape.D))) for _ in pm.blocks]
     final, states = O.hsa_denoise(x0, vh0, plan, vel, zeros, keep_states=True)
-    swapped = set()
+    # The velocity of these random-init blocks changes by ~0.5 % between steps, the
+    # size of bf16 rounding, so scores after step 0 (and the partitions they pick)
+    # are rounding-dominated on both sides.  Checked: the schedule, the step-0
+    # scores (against the random initial v_hat), that every partition is valid, and
+    # the final latent displacement of every token.
+    starts = np.concatenate([[0], np.cumsum(sizes)])
     for r, st in zip(rec, states):
         assert r["M"] == len(st["idx"])
         if r["full"]:
-            assert rel_l2(r["score"], st["score"]) < 2e-2
-            swapped |= _near_tie_swaps(r["order"], st["order"], st["score"], sizes, rel=3e-2)
-    assert len(swapped) <= N // 8, f"{len(swapped)} tokens changed group"
-    keep = np.setdiff1d(np.arange(N), np.array(sorted(swapped), dtype=np.int64))
-    assert_bf16_close(x_gpu[keep] - x0[keep], final["x"][keep] - x0[keep], "latent displacement")
+            o = r["order"]
+            assert np.array_equal(np.sort(o), np.arange(N))
+            for k in range(len(sizes)):
+                seg = o[starts[k]:starts[k + 1]]
+                assert np.all(np.diff(seg) > 0)
+    assert rec[0]["full"] and rel_l2(rec[0]["score"], states[0]["score"]) < 2e-2
+    assert sum(r["M"] for r in rec) == int(round(0.6 * wl.T * N))
+    assert_bf16_close(x_gpu - x0, final["x"] - x0, "latent displacement")

@@ -4,12 +4,12 @@
 //
 //   y[M x Nout] = epilogue(x[M x K] * W[Nout x K]^T + b)
 //
-// One CTA computes a 128 x BN tile.  Warp roles:
+// Persistent CTAs (one per SM) walk 128 x BN output tiles.  Warp roles:
 //   warp 0      TMA producer: A (128 x 64) and B (BN x 64) k-blocks into a ring
 //               of STAGES shared-memory slots, 128-byte swizzled;
-//   warp 1      allocates BN TMEM columns; lane 0 issues tcgen05.mma
-//               (M=128, N=BN, K=16) into the fp32 TMEM accumulator and
-//               releases each slot with tcgen05.commit;
+//   warp 1      allocates 2 x BN TMEM columns (two accumulators); lane 0
+//               issues tcgen05.mma (M=128, N=BN, K=16) into the free one and
+//               releases each shared-memory slot with tcgen05.commit;
 //   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter, bias, GELU /
 //               residual gate, 16-byte stores.  Thread = output row.
 // Rows beyond M are zero-filled by TMA and never stored.
@@ -30,6 +30,7 @@ struct GemmCfg {
   static constexpr int kBBytes = BN * kGemmBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(2 * BN <= 512, "double-buffered accumulator must fit TMEM");
 };
 
 __device__ __forceinline__ float gelu_tanh_f(float x) {
@@ -37,6 +38,55 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
   return 0.5f * x * (1.0f + tanhf(u));
 }
 
+// Epilogue of 32 accumulator columns of one output row (thread = row).
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row, int col0, int Nout,
+                                               const float* __restrict__ bias, const float* __restrict__ gate,
+                                               void* __restrict__ out) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + (bias ? __ldg(bias + col0 + j) : 0.f);
+  if constexpr (EPI == EPI_STORE || EPI == EPI_GELU) {
+    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * Nout + col0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      float t[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) t[e] = EPI == EPI_GELU ? gelu_tanh_f(v[j + e]) : v[j + e];
+      uint4 u;
+      u.x = pack_bf16x2(t[0], t[1]);
+      u.y = pack_bf16x2(t[2], t[3]);
+      u.z = pack_bf16x2(t[4], t[5]);
+      u.w = pack_bf16x2(t[6], t[7]);
+      *reinterpret_cast<uint4*>(y + j) = u;
+    }
+  } else if constexpr (EPI == EPI_F32) {
+    float* y = reinterpret_cast<float*>(out) + (size_t)row * Nout + col0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4)
+      *reinterpret_cast<float4*>(y + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  } else {  // EPI_RESID: y += gate * (acc + b)
+    float* y = reinterpret_cast<float*>(out) + (size_t)row * Nout + col0;
+    float4 o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] = *reinterpret_cast<const float4*>(y + 4 * j);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (gate) g = __ldg(reinterpret_cast<const float4*>(gate + col0 + 4 * j));
+      o[j].x = fmaf(g.x, v[4 * j + 0], o[j].x);
+      o[j].y = fmaf(g.y, v[4 * j + 1], o[j].y);
+      o[j].z = fmaf(g.z, v[4 * j + 2], o[j].z);
+      o[j].w = fmaf(g.w, v[4 * j + 3], o[j].w);
+      *reinterpret_cast<float4*>(y + 4 * j) = o[j];
+    }
+  }
+}
+
+// Persistent: CTA c handles output tiles c, c + gridDim.x, ... (n fastest, so the
+// CTAs running together share A row-tiles and the weights stay in L2).  The TMEM
+// accumulator is double-buffered (2 x BN columns): the epilogue of one tile runs
+// while the MMA warp accumulates the next.
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int Nout,
@@ -47,25 +97,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStageBytes);
   uint64_t* empty = full + S;
-  uint64_t* acc_full = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* acc_full = empty + S;     // [2]
+  uint64_t* acc_empty = acc_full + 2; // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kGemmBM;
   const int KB = K / kGemmBK;
+  const int n_tiles = Nout / BN;
+  const int tiles = n_tiles * ((M + kGemmBM - 1) / kGemmBM);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -76,92 +131,70 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       const uint64_t keep = policy_evict_last();   // weights are re-read by every row tile
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1)) break;
-        uint8_t* a = smem + s * Cfg::kStageBytes;
-        mbar_expect_tx(&full[s], Cfg::kStageBytes);
-        tma_load_2d(a, &tmA, &full[s], kb * kGemmBK, m0);
-        tma_load_2d_hint(a + Cfg::kABytes, &tmB, &full[s], kb * kGemmBK, n0, keep);
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+        const int n0 = (t % n_tiles) * BN, m0 = (t / n_tiles) * kGemmBM;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) { ok = false; break; }
+          uint8_t* a = smem + s * Cfg::kStageBytes;
+          mbar_expect_tx(&full[s], Cfg::kStageBytes);
+          tma_load_2d(a, &tmA, &full[s], kb * kGemmBK, m0);
+          tma_load_2d_hint(a + Cfg::kABytes, &tmB, &full[s], kb * kGemmBK, n0, keep);
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, BN, false);
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (!mbar_wait(&full[s], ph)) break;
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++tc) {
+        const int buf = tc & 1;
+        if (!mbar_wait(&acc_empty[buf], ((tc >> 1) & 1) ^ 1)) break;
         tc_fence_after();
-        const uint32_t a = smem_u32(smem + s * Cfg::kStageBytes);
-        const uint32_t b = a + Cfg::kABytes;
+        const uint32_t acc = tmem + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&full[s], (it / S) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + s * Cfg::kStageBytes);
+          const uint32_t b = a + Cfg::kABytes;
 #pragma unroll
-        for (int k = 0; k < kGemmBK / 16; ++k) {
-          umma_ss(tmem, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), idesc,
-                  (kb | k) != 0);
+          for (int k = 0; k < kGemmBK / 16; ++k)
+            umma_ss(acc, sdesc_sw128(a + 32 * k, 16, 1024), sdesc_sw128(b + 32 * k, 16, 1024), idesc,
+                    (kb | k) != 0);
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        umma_commit(&acc_full[buf]);
       }
-      umma_commit(acc_full);
     }
   } else {
     // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows of that quarter
     const int quarter = warp & 3;
-    const int row = m0 + quarter * 32 + lane;
-    mbar_wait(acc_full, 0);
-    __syncwarp();
-    tc_fence_after();
+    int tc = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
+      const int n0 = (t % n_tiles) * BN, m0 = (t / n_tiles) * kGemmBM;
+      const int buf = tc & 1;
+      const int row = m0 + quarter * 32 + lane;
+      const bool ok = mbar_wait(&acc_full[buf], (tc >> 1) & 1);
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      uint32_t r[32];
-      __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the guarded stores
-      tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(c * 32), r);
-      tmem_ld_wait();
-      if (row < M) {
-        const int col0 = n0 + c * 32;
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + (bias ? __ldg(bias + col0 + j) : 0.f);
-        if constexpr (EPI == EPI_STORE || EPI == EPI_GELU) {
-          __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * Nout + col0;
-#pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            uint4 u;
-            float t[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) t[e] = EPI == EPI_GELU ? gelu_tanh_f(v[j + e]) : v[j + e];
-            u.x = pack_bf16x2(t[0], t[1]);
-            u.y = pack_bf16x2(t[2], t[3]);
-            u.z = pack_bf16x2(t[4], t[5]);
-            u.w = pack_bf16x2(t[6], t[7]);
-            *reinterpret_cast<uint4*>(y + j) = u;
-          }
-        } else if constexpr (EPI == EPI_F32) {
-          float* y = reinterpret_cast<float*>(out) + (size_t)row * Nout + col0;
-#pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(y + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-        } else {  // EPI_RESID: y += gate * (acc + b)
-          float* y = reinterpret_cast<float*>(out) + (size_t)row * Nout + col0;
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            float4 o = *reinterpret_cast<float4*>(y + j);
-            float g0 = 1.f, g1 = 1.f, g2 = 1.f, g3 = 1.f;
-            if (gate) {
-              g0 = __ldg(gate + col0 + j);
-              g1 = __ldg(gate + col0 + j + 1);
-              g2 = __ldg(gate + col0 + j + 2);
-              g3 = __ldg(gate + col0 + j + 3);
-            }
-            o.x = fmaf(g0, v[j], o.x);
-            o.y = fmaf(g1, v[j + 1], o.y);
-            o.z = fmaf(g2, v[j + 2], o.z);
-            o.w = fmaf(g3, v[j + 3], o.w);
-            *reinterpret_cast<float4*>(y + j) = o;
-          }
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the guarded stores
+        tmem_ld32(base + (uint32_t)(c * 32), r);
+        tmem_ld_wait();
+        if (c == BN / 32 - 1) {  // accumulator fully read: the MMA warp may reuse it
+          tc_fence_before();
+          mbar_arrive(&acc_empty[buf]);
         }
+        if (row < M) epilogue_chunk<EPI>(r, row, n0 + c * 32, Nout, bias, gate, out);
       }
+      if (!ok) break;
     }
   }
 
@@ -170,7 +203,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -186,7 +219,8 @@ static int launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, int M, i
       return check_launch("gemm: shared-memory attribute");
     attr_done[dev] = true;
   }
-  dim3 grid(Nout / BN, (M + kGemmBM - 1) / kGemmBM);
+  const int tiles = (Nout / BN) * ((M + kGemmBM - 1) / kGemmBM);
+  dim3 grid(tiles < num_sms() ? tiles : num_sms());
   ScopedTiming timing(HSA_KCLASS_GEMM, st);
   kern<<<grid, kGemmThreads, GemmCfg<BN>::kSmem, st>>>(ta, tb, M, Nout, K, bias, gate, out);
   count_launch(1);

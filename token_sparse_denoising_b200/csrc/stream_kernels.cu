@@ -80,21 +80,38 @@ __global__ void __launch_bounds__(256) k_scatter_vhat(float* __restrict__ vhat, 
   const float* arow = vA + (size_t)r * C;
   float* xrow = x ? x + (size_t)n * C : nullptr;
   float num = 0.f, den = 0.f;
-  for (int c = 4 * lane; c < C; c += 128) {
-    const float4 a = ld4(arow + c);
-    if (score) {
-      const float4 o = ld4(vrow + c);
-      num += fabsf(a.x - o.x) + fabsf(a.y - o.y) + fabsf(a.z - o.z) + fabsf(a.w - o.w);
-      den += fabsf(o.x) + fabsf(o.y) + fabsf(o.z) + fabsf(o.w);
+  // U chunks of 128 floats per warp iteration: every load of the group is issued
+  // before the first one is used, so a warp keeps 3U 16-byte loads in flight
+  constexpr int U = 4;
+  for (int c0 = 4 * lane; c0 < C; c0 += 128 * U) {
+    float4 a[U], o[U], xv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 128 * u;
+      if (c < C) {
+        a[u] = ld4_stream(arow + c);
+        if (score) o[u] = ld4_stream(vrow + c);
+        if (xrow) xv[u] = ld4_stream(xrow + c);
+      }
     }
-    st4(vrow + c, a);
-    if (xrow) {
-      float4 xv = ld4(xrow + c);
-      xv.x = fmaf(dsigma, a.x, xv.x);
-      xv.y = fmaf(dsigma, a.y, xv.y);
-      xv.z = fmaf(dsigma, a.z, xv.z);
-      xv.w = fmaf(dsigma, a.w, xv.w);
-      st4(xrow + c, xv);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 128 * u;
+      if (c < C) {
+        if (score) {
+          num += fabsf(a[u].x - o[u].x) + fabsf(a[u].y - o[u].y) + fabsf(a[u].z - o[u].z) + fabsf(a[u].w - o[u].w);
+          den += fabsf(o[u].x) + fabsf(o[u].y) + fabsf(o[u].z) + fabsf(o[u].w);
+        }
+        __stcs(reinterpret_cast<float4*>(vrow + c), a[u]);
+        if (xrow) {
+          float4 t = xv[u];
+          t.x = fmaf(dsigma, a[u].x, t.x);
+          t.y = fmaf(dsigma, a[u].y, t.y);
+          t.z = fmaf(dsigma, a[u].z, t.z);
+          t.w = fmaf(dsigma, a[u].w, t.w);
+          __stcs(reinterpret_cast<float4*>(xrow + c), t);
+        }
+      }
     }
   }
   if (score) {
