@@ -53,6 +53,9 @@ def parse():
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--mode", choices=["step", "loop", "sweep", "wan14"], default="step",
+                   help="step: the headline line; loop: 30-block Wan-1.3B loop, HSA vs uniform 40 steps; "
+                        "sweep: attention + Euler kernel sweep; wan14: Wan-14B block active-fraction sweep")
     return p.parse_args()
 
 
@@ -287,6 +290,107 @@ def run_gpu(args, rank, world, barrier, allmax):
     return out
 
 
+# ---------------------------------------------------------------- extra measurement modes
+
+def run_loop(args):
+    """Full Wan-1.3B-shaped loop: latent 16x21x60x104 patchified 1x2x2 (N=32760, C=64), 30 blocks,
+    T=40; HSA with budgets {40,20,10} sized 25/25/50 % and m=4 against the uniform 40-step run."""
+    import torch
+    from token_sparse_denoising_b200 import hsa, pipeline
+    hsa.load()
+    wl = S.WAN13_LOOP
+    N = wl.grid.N
+    pm = S.patch_model_weights(wl.seed, wl.shape, wl.C, wl.n_blocks, True)
+    pos = S.token_positions(wl.grid)
+    ctx = S.normal(wl.seed * 10 + 3, (wl.shape.ctx_len, wl.shape.D), 1.0, True)
+    x0, vh0 = S.normal(wl.seed * 10 + 1, (N, wl.C)), S.normal(wl.seed * 10 + 2, (N, wl.C))
+    model = pipeline.PatchModel(pm, pos, N, bf16=True, ctx=ctx)
+    out = {"mode": "loop", "workload": f"{wl.name}: 30 blocks D=1536 H=12 F=8960 ctx=512, T=40, m=4, shift 5"}
+    for name, budgets, fracs in (("hsa", wl.budgets, wl.fracs), ("uniform", (wl.T,), (1.0,))):
+        sizes = S.group_sizes(N, fracs)
+        run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift)
+        run.step()                                     # warm-up iteration (not timed)
+        run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        run.run()
+        b.record()
+        b.synchronize()
+        assert hsa.device_status() == 0
+        out[name] = {"ms": round(a.elapsed_time(b), 1), "token_steps": int(run.n_active.sum()),
+                     "active_fraction": round(float(run.n_active.sum()) / (wl.T * N), 4)}
+    out["speedup"] = round(out["uniform"]["ms"] / out["hsa"]["ms"], 3)
+    return out
+
+
+def run_sweep(args):
+    """Attention at N in {8190, 32760, 75600} x |A|/N in {1, .5, .25, .125} (12 heads, random active rows)
+    and the Euler update on N x 64 fp32 latents."""
+    import torch
+    from token_sparse_denoising_b200 import hsa
+    hsa.load()
+    peak_burst = load_peaks()[1]
+    hbm = load_peaks()[2]
+    res = {"mode": "sweep", "attention": [], "euler": []}
+    for N in (8190, 32760, 75600):
+        k = torch.randn((N, 1536), device="cuda").to(torch.bfloat16)
+        v = torch.randn((N, 1536), device="cuda").to(torch.bfloat16)
+        for f in (1.0, 0.5, 0.25, 0.125):
+            M = S.active_fraction_rows(N, f)
+            q = torch.randn((M, 1536), device="cuda").to(torch.bfloat16)
+            o = torch.empty_like(q)
+            reps = 5
+            for _ in range(2):
+                hsa.attention(q, k, v, 12, o)
+            ms = time_device(lambda: hsa.attention(q, k, v, 12, o), reps, lambda: None) / reps
+            tf = 4.0 * M * N * 128 * 12 / (ms * 1e-3) / 1e12
+            res["attention"].append({"N": N, "frac": f, "M": M, "ms": round(ms, 4), "tflops": round(tf, 1),
+                                     "frac_of_burst_peak": round(tf / peak_burst, 3)})
+        x = torch.randn((N, 64), device="cuda")
+        vh = torch.randn((N, 64), device="cuda")
+        flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda")   # > L2: evict between reps
+        times = []
+        for _ in range(5):
+            flush.zero_()
+            times.append(time_device(lambda: hsa.euler_update(x, vh, None, None, -0.025), 1, lambda: None))
+        ms = min(times)
+        res["euler"].append({"N": N, "C": 64, "ms": round(ms, 5), "bytes": 12 * N * 64,
+                             "gbs": round(12 * N * 64 / (ms * 1e-3) / 1e9, 1),
+                             "frac_of_hbm": round(12 * N * 64 / (ms * 1e-3) / 1e9 / hbm, 3)})
+    return res
+
+
+def run_wan14(args):
+    """Wan-14B block (D=5120, 40 heads, FFN 13824, no context) at |A|/N in {1, .5, .25, .125},
+    contiguous and scattered active sets: layer-step ms."""
+    import torch
+    from token_sparse_denoising_b200 import hsa
+    hsa.load()
+    grid, shape = S.WAN13_GRID, S.WAN14_BLOCK
+    N, D = grid.N, shape.D
+    w = hsa.LayerWeights(S.block_weights(4, shape, True), "cuda", True)
+    kc = torch.randn((N, D), device="cuda").to(torch.bfloat16)
+    vc = torch.randn((N, D), device="cuda").to(torch.bfloat16)
+    x = torch.randn((N, D), device="cuda")
+    pos = torch.from_numpy(S.token_positions(grid)).cuda()
+    ws = torch.empty(hsa.layer_step_workspace_size(N, D, shape.F, hsa.HSA_BF16), dtype=torch.uint8, device="cuda")
+    xA = torch.empty((N, D), device="cuda")
+    res = {"mode": "wan14", "workload": "wan14b-block N=32760 D=5120 H=40 F=13824", "points": []}
+    for f in (1.0, 0.5, 0.25, 0.125):
+        M = S.active_fraction_rows(N, f)
+        for pattern in ("contiguous", "scattered"):
+            idx = torch.from_numpy((S.contiguous_mask if pattern == "contiguous" else S.scattered_mask)(46, N, M)).cuda()
+            fn = lambda: hsa.layer_step(w, kc, vc, xA[:M], idx, pos, ws, x_src=x)
+            fn()
+            ms = time_device(fn, 3, lambda: None) / 3
+            flops = 4.0 * M * N * 128 * 40 + 2.0 * M * (3 * D * D + D * D + 2 * D * shape.F)
+            res["points"].append({"frac": f, "pattern": pattern, "M": M, "ms": round(ms, 3),
+                                  "tflops": round(flops / (ms * 1e-3) / 1e12, 1)})
+    assert hsa.device_status() == 0
+    return res
+
+
 # ---------------------------------------------------------------- the oracle on the host cores
 
 ORACLE_ROWS = 32        # attention / O / cross / FFN query rows per sample
@@ -383,6 +487,11 @@ def main():
 
     import torch
     torch.cuda.set_device(local)
+    if args.mode != "step":
+        if rank == 0:
+            fn = {"loop": run_loop, "sweep": run_sweep, "wan14": run_wan14}[args.mode]
+            print(json.dumps(fn(args)), flush=True)
+        return 0
     dist = None
     if world > 1:
         import datetime

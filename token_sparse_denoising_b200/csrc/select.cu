@@ -85,9 +85,18 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += kSelectThreads) hist[i] = 0;
       __syncthreads();
-      for (int n = tid; n < N; n += kSelectThreads) {
-        const uint32_t ik = ~score_key(score[n]);
-        if ((ik & mask) == prefix) atomicAdd(&hist[(ik >> shift) & 255u], 1u);
+      // warp-aggregated histogram: lanes with the same bin add once (scores share few
+      // exponent bytes, so plain per-lane atomics would serialise on one address)
+      const int lane = tid & 31;
+      for (int base = 0; base < N; base += kSelectThreads) {
+        const int n = base + tid;
+        uint32_t bin = 256u + (uint32_t)lane;          // unique non-bin value when inactive
+        if (n < N) {
+          const uint32_t ik = ~score_key(score[n]);
+          if ((ik & mask) == prefix) bin = (ik >> shift) & 255u;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
       }
       __syncthreads();
       if (tid == 0) {
