@@ -157,6 +157,28 @@ int hsa_context_kv(const void* d_ctx, int L, int D, int dtype, const void* d_w_k
                    const float* d_b_kv2, const float* d_g_k2, void* d_k2, void* d_v2, void* d_ws,
                    size_t ws_bytes, void* stream);
 
+/* The same projection for callers that cannot allocate device memory.  The paper
+ * has no counterpart: this entry exists for embedders that may not call cudaMalloc
+ * (or any allocating library routine) where they need the context keys/values, for
+ * instance a runtime whose device memory budget is fixed at start-up, or code on a
+ * path where an allocation would synchronise the device.  Instead of a caller
+ * workspace it uses a scratch array built into the library: 8 MiB
+ * (hsa_context_kv_noalloc_max_bytes()), held by every GPU that loads libhsa until
+ * the process exits.  It allocates nothing.
+ *   - Arguments as hsa_context_kv, without the workspace.  L x 2D x 4 bytes must not
+ *     exceed the scratch size, else HSA_EINVAL (e.g. L = 512 fits up to D = 2048).
+ *   - The first call on a device looks up the scratch's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call shares the one scratch array and leaves its contents behind; the
+ *     projection writes each scratch element before reading it, so no clearing is
+ *     needed.  Calls whose GPU work overlaps (other streams, other host threads on
+ *     the same device) race on the scratch: order them on one stream. */
+size_t hsa_context_kv_noalloc_max_bytes(void);
+int hsa_context_kv_noalloc(const void* d_ctx, int L, int D, int dtype, const void* d_w_kv2,
+                           const float* d_b_kv2, const float* d_g_k2, void* d_k2, void* d_v2,
+                           void* stream);
+
 /* One block on the active rows of iteration i (§2.2):
  *   X = x_A (M x D float32, the residual stream of the active tokens, in/out);
  *   h = LN(X)(1 + mod1) + mod0;  [q k v] = h W_qkv^T + b_qkv;

@@ -8,3 +8,4 @@
 #include "attn_tc.cu"
 #include "simt_f32.cu"
 #include "api.cu"
+#include "noalloc.cu"

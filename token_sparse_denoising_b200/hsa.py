@@ -50,6 +50,8 @@ _SIGS = {
     "hsa_euler_update": (i32, [vp, vp, vp, vp, i32, i32, i32, f32, vp, vp]),
     "hsa_context_kv_workspace_size": (sz, [i32, i32]),
     "hsa_context_kv": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
+    "hsa_context_kv_noalloc_max_bytes": (sz, []),
+    "hsa_context_kv_noalloc": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
     "hsa_layer_step_workspace_size": (sz, [i32, i32, i32, i32]),
     "hsa_layer_step": (i32, [C.POINTER(LayerWeightsC), vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, i32, vp, sz, vp]),
     "hsa_attention": (i32, [vp, i32, vp, vp, i32, i32, i32, vp, vp]),
@@ -202,6 +204,13 @@ def context_kv(ctx, w_kv2, b_kv2, g_k2, k2, v2, ws, stream=None):
     _check(lib().hsa_context_kv(_ptr(ctx), L, D, _dtype_code(ctx), _ptr(w_kv2), _ptr(b_kv2), _ptr(g_k2), _ptr(k2),
                                 _ptr(v2), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "hsa_context_kv")
+
+
+def context_kv_noalloc(ctx, w_kv2, b_kv2, g_k2, k2, v2, stream=None):
+    """hsa_context_kv without a workspace: scratch comes from an array built into libhsa."""
+    L, D = ctx.shape
+    _check(lib().hsa_context_kv_noalloc(_ptr(ctx), L, D, _dtype_code(ctx), _ptr(w_kv2), _ptr(b_kv2), _ptr(g_k2),
+                                        _ptr(k2), _ptr(v2), _stream(stream)), "hsa_context_kv_noalloc")
 
 
 def layer_step_workspace_size(M: int, D: int, F: int, dtype: int) -> int:
