@@ -121,7 +121,7 @@ extern "C" int hsa_euler_update(float* d_x, float* d_vhat, const float* d_vA, co
     HSA_TRY(check_launch("v_hat scatter launch"));
   }
   const size_t n4 = (size_t)N * C / 4;
-  const size_t want = (n4 + 255) / 256;
+  const size_t want = (n4 + 1023) / 1024;   // 4 float4 per thread per iteration
   const size_t cap = (size_t)num_sms() * 8;
   k_euler<<<(unsigned)(want < cap ? want : cap), 256, 0, st>>>(d_x, d_vhat, n4, dsigma);
   count_launch(1);

@@ -11,7 +11,9 @@
 //               issues tcgen05.mma (M=128, N=BN, K=16) into the free one and
 //               releases each shared-memory slot with tcgen05.commit;
 //   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter, bias, GELU /
-//               residual gate, 16-byte stores.  Thread = output row.
+//               residual gate.  Thread = output row.  bf16 outputs are staged per
+//               warp as 32 x 32 sub-tiles in shared memory and written by TMA stores;
+//               the fp32 residual update reads and writes rows directly.
 // Rows beyond M are zero-filled by TMA and never stored.
 #include "tcgen05.cuh"
 
@@ -29,7 +31,9 @@ struct GemmCfg {
   static constexpr int kABytes = kGemmBM * kGemmBK * 2;   // 16 KB
   static constexpr int kBBytes = BN * kGemmBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  // epilogue staging for the bf16 outputs: 4 warps x 2 buffers x (32 rows x 64 bytes)
+  static constexpr int kStageOutBytes = 4 * 2 * 2048;
+  static constexpr int kSmem = kStages * kStageBytes + kStageOutBytes + 1024 /*align*/ + 256 /*barriers*/;
   static_assert(2 * BN <= 512, "double-buffered accumulator must fit TMEM");
 };
 
@@ -89,13 +93,16 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row,
 // while the MMA warp accumulates the next.
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int Nout,
-              int K, const float* __restrict__ bias, const float* __restrict__ gate, void* __restrict__ out) {
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmY, int M, int Nout, int K, const float* __restrict__ bias,
+              const float* __restrict__ gate, void* __restrict__ out) {
   using Cfg = GemmCfg<BN>;
   constexpr int S = Cfg::kStages;
+  constexpr bool kTmaOut = (EPI == EPI_STORE || EPI == EPI_GELU);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStageBytes);
+  uint8_t* stage_out = smem + S * Cfg::kStageBytes;   // 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(stage_out + Cfg::kStageOutBytes);
   uint64_t* empty = full + S;
   uint64_t* acc_full = empty + S;     // [2]
   uint64_t* acc_empty = acc_full + 2; // [2]
@@ -118,6 +125,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (kTmaOut) prefetch_tmap(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 2 * BN);
@@ -173,7 +181,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows of that quarter
     const int quarter = warp & 3;
-    int tc = 0;
+    uint8_t* my_out = stage_out + (warp - 2) * 2 * 2048;   // this warp's two 32 x 32 bf16 buffers
+    int tc = 0, nchunk = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
       const int n0 = (t % n_tiles) * BN, m0 = (t / n_tiles) * kGemmBM;
       const int buf = tc & 1;
@@ -183,7 +192,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < BN / 32; ++c, ++nchunk) {
         uint32_t r[32];
         __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the guarded stores
         tmem_ld32(base + (uint32_t)(c * 32), r);
@@ -192,10 +201,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_before();
           mbar_arrive(&acc_empty[buf]);
         }
-        if (row < M) epilogue_chunk<EPI>(r, row, n0 + c * 32, Nout, bias, gate, out);
+        if constexpr (kTmaOut) {
+          // stage the warp's 32 x 32 sub-tile (64-byte swizzle: chunk k of row r at k ^ ((r>>1)&3),
+          // conflict-free for thread-per-row writes) and store it with one TMA copy; rows
+          // beyond M are clipped by the tensor map
+          uint8_t* sb = my_out + (nchunk & 1) * 2048;
+          if (lane == 0) bulk_wait_group_read<1>();   // the store that last read sb is done
+          __syncwarp();
+          const int col0 = n0 + c * 32;
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float v0 = __uint_as_float(r[2 * j]) + (bias ? __ldg(bias + col0 + 2 * j) : 0.f);
+            float v1 = __uint_as_float(r[2 * j + 1]) + (bias ? __ldg(bias + col0 + 2 * j + 1) : 0.f);
+            if (EPI == EPI_GELU) {
+              v0 = gelu_tanh_f(v0);
+              v1 = gelu_tanh_f(v1);
+            }
+            w[j] = pack_bf16x2(v0, v1);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(sb + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, sb, col0, m0 + quarter * 32);
+            bulk_commit_group();
+          }
+        } else {
+          if (row < M) epilogue_chunk<EPI>(r, row, n0 + c * 32, Nout, bias, gate, out);
+        }
       }
       if (!ok) break;
     }
+    if (kTmaOut && lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();
@@ -208,8 +249,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 template <int BN, int EPI>
-static int launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, int M, int Nout, int K, const float* bias,
-                          const float* gate, void* out, cudaStream_t st) {
+static int launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, int M, int Nout,
+                          int K, const float* bias, const float* gate, void* out, cudaStream_t st) {
   auto kern = k_gemm_tc<BN, EPI>;
   static bool attr_done[64] = {false};
   int dev = 0;
@@ -222,7 +263,7 @@ static int launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, int M, i
   const int tiles = (Nout / BN) * ((M + kGemmBM - 1) / kGemmBM);
   dim3 grid(tiles < num_sms() ? tiles : num_sms());
   ScopedTiming timing(HSA_KCLASS_GEMM, st);
-  kern<<<grid, kGemmThreads, GemmCfg<BN>::kSmem, st>>>(ta, tb, M, Nout, K, bias, gate, out);
+  kern<<<grid, kGemmThreads, GemmCfg<BN>::kSmem, st>>>(ta, tb, ty, M, Nout, K, bias, gate, out);
   count_launch(1);
   return check_launch("gemm_tc launch");
 }
@@ -236,9 +277,14 @@ static int launch_gemm_epi(const void* A, int M, int K, const void* W, int Nout,
   if (rc) return rc;
   rc = make_tmap_2d(&tb, W, true, (uint64_t)K, (uint64_t)Nout, (uint64_t)K * 2, kGemmBK, (uint32_t)BN, true);
   if (rc) return rc;
-  if (BN == 256) return launch_gemm_bn<256, EPI>(ta, tb, M, Nout, K, bias, gate, out, st);
-  if (BN == 128) return launch_gemm_bn<128, EPI>(ta, tb, M, Nout, K, bias, gate, out, st);
-  return launch_gemm_bn<64, EPI>(ta, tb, M, Nout, K, bias, gate, out, st);
+  CUtensorMap ty = tb;   // unused unless the output is bf16
+  if (EPI == EPI_STORE || EPI == EPI_GELU) {
+    rc = make_tmap_2d_sw64(&ty, out, true, (uint64_t)Nout, (uint64_t)M, (uint64_t)Nout * 2, 32, 32);
+    if (rc) return rc;
+  }
+  if (BN == 256) return launch_gemm_bn<256, EPI>(ta, tb, ty, M, Nout, K, bias, gate, out, st);
+  if (BN == 128) return launch_gemm_bn<128, EPI>(ta, tb, ty, M, Nout, K, bias, gate, out, st);
+  return launch_gemm_bn<64, EPI>(ta, tb, ty, M, Nout, K, bias, gate, out, st);
 }
 
 // Host entry used by every bf16 linear layer.  Shapes are validated here.

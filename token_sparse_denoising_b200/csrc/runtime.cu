@@ -59,8 +59,9 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-int make_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
-                 uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+static int make_tmap_2d_impl(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+                             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                             CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return set_error(HSA_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
   if (!aligned16(base) || (row_stride_bytes & 15u))
@@ -71,7 +72,7 @@ int make_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, 
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     char buf[160];
@@ -80,6 +81,18 @@ int make_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, 
     return set_error(HSA_ECUDA, buf);
   }
   return HSA_OK;
+}
+
+int make_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+                 uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  return make_tmap_2d_impl(map, base, bf16, inner, outer, row_stride_bytes, box_inner, box_outer,
+                           swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+int make_tmap_2d_sw64(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  return make_tmap_2d_impl(map, base, bf16, inner, outer, row_stride_bytes, box_inner, box_outer,
+                           CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 // ------------------------------------------------------------------ per-kernel timing

@@ -18,6 +18,9 @@ int num_sms();
 // (bf16 or f32), rows `row_stride_bytes` apart, boxes of box_outer x box_inner.
 int make_tmap_2d(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
                  uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+// Same with the 64-byte swizzle (boxes whose inner extent is 64 bytes).
+int make_tmap_2d_sw64(CUtensorMap* map, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
 
 // Records a CUDA event pair around the launches made while it is alive, when
 // timing is enabled (hsa_timing_enable); otherwise does nothing.

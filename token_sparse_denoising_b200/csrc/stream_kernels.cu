@@ -46,11 +46,30 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
 }
 
 // ------------------------------------------------------------------ §2.3 cached Euler
-// x[e] += dsigma * v_hat[e] for every element; n4 float4 groups, grid-stride.
+// x[e] += dsigma * v_hat[e] for every element; n4 float4 groups, grid-stride with
+// U groups per thread per iteration, all loaded before any is used.
 __global__ void __launch_bounds__(256) k_euler(float* __restrict__ x, const float* __restrict__ vhat, size_t n4,
                                                float dsigma) {
+  constexpr int U = 4;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + (U - 1) * stride < n4; i += U * stride) {
+    float4 xv[U], v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      xv[u] = ld4_stream(x + 4 * (i + u * stride));
+      v[u] = ld4_stream(vhat + 4 * (i + u * stride));
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      xv[u].x = fmaf(dsigma, v[u].x, xv[u].x);
+      xv[u].y = fmaf(dsigma, v[u].y, xv[u].y);
+      xv[u].z = fmaf(dsigma, v[u].z, xv[u].z);
+      xv[u].w = fmaf(dsigma, v[u].w, xv[u].w);
+      __stcs(reinterpret_cast<float4*>(x + 4 * (i + u * stride)), xv[u]);
+    }
+  }
+  for (; i < n4; i += stride) {
     float4 xv = ld4_stream(x + 4 * i);
     const float4 v = ld4_stream(vhat + 4 * i);
     xv.x = fmaf(dsigma, v.x, xv.x);
