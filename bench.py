@@ -481,6 +481,28 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- main
 
+def collectives(dist, device):
+    """Barrier and max-over-ranks of a float; plain pass-throughs on one process.
+
+    `dist` is torch.distributed after init_process_group (NCCL on the GPUs, gloo in the
+    CPU tests) or None.  Every rank calls both in the same order.
+    """
+    import torch
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def allmax(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, allmax
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -506,16 +528,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
 
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def allmax(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, allmax = collectives(dist, "cuda")
 
     try:
         out = run_gpu(args, rank, world, barrier, allmax)

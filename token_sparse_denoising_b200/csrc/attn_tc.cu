@@ -42,11 +42,6 @@ constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 #define HSA_ATTN_POLY_PER8 0
 #endif
 constexpr int kPolyPer8 = HSA_ATTN_POLY_PER8;
-// 3: row max shared by the two column halves (k_attn_tc); 4: independent halves with P
-// in shared memory (k_attn_tc4).
-#ifndef HSA_ATTN_VARIANT
-#define HSA_ATTN_VARIANT 3
-#endif
 
 struct AttnShared {
   uint64_t q_full;
@@ -313,276 +308,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------------------------------------
-// k_attn_tc4: the same tiling with independent column halves.  Each softmax thread owns
-// 64 of a tile's 128 key columns for its row and keeps its own running max, row sum and
-// O accumulator (O_L for the left key half, O_R for the right one), so the two warps that
-// share a lane quarter never wait for each other inside the key loop.  P goes through
-// shared memory (128-byte swizzled, K-major A operand of an SS-MMA):
-//   O_L += P[:, 0:64] V[0:64, :],  O_R += P[:, 64:128] V[64:128, :]
-// and the halves are merged once at the end:
-//   o = (O_L 2^(m_L - m) + O_R 2^(m_R - m)) / (l_L 2^(m_L - m) + l_R 2^(m_R - m)).
-// TMEM columns: S0 [0,128) S1 [128,256) O_L [256,384) O_R [384,512).
-// Shared memory: Q | K x2 | V x2 | P x2 (32 KB each) | barriers.
-constexpr int kA4KSlots = 2;
-constexpr int kA4VSlots = 2;
-
-struct Attn4Shared {
-  uint64_t q_full;
-  uint64_t k_full[kA4KSlots], k_empty[kA4KSlots];
-  uint64_t v_full[kA4VSlots], v_empty[kA4VSlots];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2][2], pv_done[2][2];   // [P buffer][column half]
-  uint32_t tmem;
-};
-constexpr int kAttn4Smem = kTileBytes * (1 + kA4KSlots + kA4VSlots + 2) + 1024 + (int)sizeof(Attn4Shared);
-
-__global__ void __launch_bounds__(kAttnThreads, 1)
-    k_attn_tc4(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, int M, int L, int H, __nv_bfloat16* __restrict__ O) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kTileBytes;
-  uint8_t* sV = sK + kA4KSlots * kTileBytes;
-  uint8_t* sP = sV + kA4VSlots * kTileBytes;              // P buffer b at b * kTileBytes; half h at + h * 16 KB
-  Attn4Shared* sh = reinterpret_cast<Attn4Shared*>(sP + 2 * kTileBytes);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kAttnBM, h = blockIdx.y;
-  const int nj = (L + kAttnBN - 1) / kAttnBN;
-
-  if (threadIdx.x == 0) {
-    mbar_init(&sh->q_full, 1);
-    for (int s = 0; s < kA4KSlots; ++s) {
-      mbar_init(&sh->k_full[s], 1);
-      mbar_init(&sh->k_empty[s], 1);
-    }
-    for (int s = 0; s < kA4VSlots; ++s) {
-      mbar_init(&sh->v_full[s], 1);
-      mbar_init(&sh->v_empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sh->s_full[b], 1);
-      mbar_init(&sh->s_free[b], 256);
-      for (int q = 0; q < 2; ++q) {
-        mbar_init(&sh->p_full[b][q], 128);
-        mbar_init(&sh->pv_done[b][q], 1);
-      }
-    }
-    fence_mbar_init();
-    prefetch_tmap(&tmQ);
-    prefetch_tmap(&tmK);
-    prefetch_tmap(&tmV);
-  }
-  if (warp == 1) {
-    tmem_alloc(&sh->tmem, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tm = sh->tmem;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      const int x0 = h * 128;
-      mbar_expect_tx(&sh->q_full, kTileBytes);
-      tma_load_2d(sQ, &tmQ, &sh->q_full, x0, m0);
-      tma_load_2d(sQ + kTileBytes / 2, &tmQ, &sh->q_full, x0 + 64, m0);
-      for (int j = 0; j < nj; ++j) {
-        const int sk = j % kA4KSlots, sv = j % kA4VSlots;
-        if (!mbar_wait(&sh->k_empty[sk], ((j / kA4KSlots) & 1) ^ 1)) break;
-        uint8_t* k = sK + sk * kTileBytes;
-        mbar_expect_tx(&sh->k_full[sk], kTileBytes);
-        tma_load_2d(k, &tmK, &sh->k_full[sk], x0, j * kAttnBN);
-        tma_load_2d(k + kTileBytes / 2, &tmK, &sh->k_full[sk], x0 + 64, j * kAttnBN);
-        if (!mbar_wait(&sh->v_empty[sv], ((j / kA4VSlots) & 1) ^ 1)) break;
-        uint8_t* v = sV + sv * kTileBytes;
-        mbar_expect_tx(&sh->v_full[sv], kTileBytes);
-        tma_load_2d(v, &tmV, &sh->v_full[sv], x0, j * kAttnBN);
-        tma_load_2d(v + kTileBytes / 2, &tmV, &sh->v_full[sv], x0 + 64, j * kAttnBN);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
-      const uint32_t q_addr = smem_u32(sQ);
-      bool ok = mbar_wait(&sh->q_full, 0);
-      auto issue_qk = [&](int j) -> bool {
-        const int sk = j % kA4KSlots, b = j & 1;
-        if (!mbar_wait(&sh->k_full[sk], (j / kA4KSlots) & 1)) return false;
-        if (j >= 2 && !mbar_wait(&sh->s_free[b], ((j - 2) >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + sk * kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-          umma_ss(tm + kColS + b * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
-                  idesc_s, kk > 0);
-        }
-        umma_commit(&sh->s_full[b]);
-        umma_commit(&sh->k_empty[sk]);
-        return true;
-      };
-      if (ok) ok = issue_qk(0);
-      for (int j = 0; ok && j < nj; ++j) {
-        if (j + 1 < nj && !issue_qk(j + 1)) break;
-        const int b = j & 1, sv = j % kA4VSlots;
-        if (!mbar_wait(&sh->v_full[sv], (j / kA4VSlots) & 1)) break;
-        const uint32_t v_addr = smem_u32(sV + sv * kTileBytes);
-        const uint32_t p_addr = smem_u32(sP + b * kTileBytes);
-        for (int q = 0; q < 2; ++q) {
-          if (!mbar_wait(&sh->p_full[b][q], (j >> 1) & 1)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            // A: P rows, keys [64q + 16kk, +16) (K-major, one 64-key swizzle atom column per half)
-            // B: V keys [64q + 16kk, +16) (MN-major, two 1024-byte atoms per 16 keys)
-            umma_ss(tm + 256 + 128 * q, sdesc_sw128(p_addr + q * (kTileBytes / 2) + kk * 32, 16, 1024),
-                    sdesc_sw128(v_addr + (4 * q + kk) * 2048, kTileBytes / 2, 1024), idesc_o, (j > 0 || kk > 0));
-          }
-          umma_commit(&sh->pv_done[b][q]);
-        }
-        if (!ok) break;
-        umma_commit(&sh->v_empty[sv]);
-      }
-    }
-  } else {
-    // ---------------------------------------------------------------- softmax warps
-    const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int row = quarter * 32 + lane;
-    const uint32_t lane_base = tm + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t o_base = lane_base + 256 + 128 * half;     // this half's O accumulator
-    const float sc = 0.12751743074680484f;                    // log2(e) / sqrt(128)
-    float m = -INFINITY, l = 0.f;
-    for (int j = 0; j < nj; ++j) {
-      const int b = j & 1;
-      mbar_wait(&sh->s_full[b], (j >> 1) & 1);
-      __syncwarp();
-      tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(lane_base + kColS + b * 128 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(sr));
-      tmem_ld32(lane_base + kColS + b * 128 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&sh->s_free[b]);
-
-      if ((j + 1) * kAttnBN > L) {
-        const int valid = L - j * kAttnBN - half * 64;
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
-      }
-      float mx8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
-#pragma unroll
-      for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-      // a half whose 64 keys all lie beyond L keeps its max (nothing to add this tile)
-      const float m_tile = sc * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                      fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      if (j == 0) {
-        m = m_tile;
-      } else {
-        const bool need = m_tile > m + 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          mbar_wait(&sh->pv_done[(j - 1) & 1][half], ((j - 1) >> 1) & 1);
-          __syncwarp();
-          tc_fence_after();
-          const float corr = need ? ex2_approx(m - m_tile) : 1.0f;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(o_base + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-            tmem_st32(o_base + c * 32, o);
-          }
-          tmem_st_wait();
-          if (need) {
-            l *= corr;
-            m = m_tile;
-          }
-        }
-      }
-      // m = -inf only if every key this half has seen so far lay beyond L (first tile, L < 64):
-      // use 0 so that 2^(-inf - 0) = 0 instead of NaN
-      const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      uint32_t pk[32];
-      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c]), sc, neg_m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + 1]), sc, neg_m));
-        rs8[(c >> 1) & 7] += p0 + p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
-      }
-      l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-      // P buffer b, this half, was last read by PV_half(j-2)
-      if (j >= 2) mbar_wait(&sh->pv_done[b][half], ((j - 2) >> 1) & 1);
-      uint8_t* prow = sP + b * kTileBytes + half * (kTileBytes / 2) + row * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)   // 16-byte chunk c of the row lands at chunk c ^ (row % 8)
-        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
-      mbar_arrive(&sh->p_full[b][half]);
-    }
-    // ---------------------------------------------------------------- merge the halves, store
-    // once the last PV MMAs are done the P buffers are free: they carry the max / sum exchange
-    mbar_wait(&sh->pv_done[(nj - 1) & 1][0], ((nj - 1) >> 1) & 1);
-    mbar_wait(&sh->pv_done[(nj - 1) & 1][1], ((nj - 1) >> 1) & 1);
-    float* xch = reinterpret_cast<float*>(sP);     // [m: half][row], then [l: half][row]
-    xch[half * 128 + row] = m;
-    xch[256 + half * 128 + row] = l;
-    named_bar_sync(1 + quarter, 64);
-    const float mL = xch[row], mR = xch[128 + row];
-    const float mx = fmaxf(mL, mR);
-    const float fL = (mL == -INFINITY) ? 0.f : ex2_approx(mL - mx);
-    const float fR = (mR == -INFINITY) ? 0.f : ex2_approx(mR - mx);
-    const float inv_l = 1.0f / (xch[256 + row] * fL + xch[384 + row] * fR);
-    const float aL = fL * inv_l, aR = fR * inv_l;
-    __syncwarp();
-    tc_fence_after();
-    const int grow = m0 + row;
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {   // this thread writes output channels [64 half + 32 c, +32)
-      uint32_t a[32], bv[32];
-      __syncwarp();
-      tmem_ld32(lane_base + 256 + half * 64 + c * 32, a);
-      tmem_ld32(lane_base + 384 + half * 64 + c * 32, bv);
-      tmem_ld_wait();
-      if (grow < M) {
-        __nv_bfloat16* dst = O + (size_t)grow * (H * 128) + h * 128 + half * 64 + c * 32;
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          float t[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) t[q] = __uint_as_float(a[e + q]) * aL + __uint_as_float(bv[e + q]) * aR;
-          uint4 u;
-          u.x = pack_bf16x2(t[0], t[1]);
-          u.y = pack_bf16x2(t[2], t[3]);
-          u.z = pack_bf16x2(t[4], t[5]);
-          u.w = pack_bf16x2(t[6], t[7]);
-          *reinterpret_cast<uint4*>(dst + e) = u;
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tm, 512);
-  }
-}
-
 int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, int H, void* O, cudaStream_t st) {
   if (M <= 0) return HSA_OK;
   if (L <= 0 || H <= 0) return set_error(HSA_EINVAL, "attention: need L > 0 and H > 0");
@@ -599,18 +324,13 @@ int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, in
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return set_error(HSA_ECUDA, "attention: device index out of range");
   if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(k_attn_tc4, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttn4Smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess)
       return check_launch("attention: shared-memory attribute");
     attr_done[dev] = true;
   }
   ScopedTiming timing(HSA_KCLASS_ATTENTION, st);
   dim3 grid((M + kAttnBM - 1) / kAttnBM, H);
-#if HSA_ATTN_VARIANT == 4
-  k_attn_tc4<<<grid, kAttnThreads, kAttn4Smem, st>>>(tq, tk, tv, M, L, H, reinterpret_cast<__nv_bfloat16*>(O));
-#else
   k_attn_tc<<<grid, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, M, L, H, reinterpret_cast<__nv_bfloat16*>(O));
-#endif
   count_launch(1);
   return check_launch("attn_tc launch");
 }

@@ -9,11 +9,15 @@
 //
 // One 1024-thread CTA (the work is a few passes over N floats):
 //   1. for each boundary c_k (k < K): radix-select, over the 32-bit order key,
-//      the element of rank c_k - 1 (4 passes of 8 bits with a shared-memory
-//      histogram), then the right index among the equal keys by a block scan;
+//      the element of rank c_k - 1 (4 passes of 8 bits; per-warp private
+//      shared-memory histograms, since scores share few exponent bytes; the
+//      top-digit pass is shared by all boundaries), then the right index among
+//      the equal keys by a block scan;
 //   2. each token's group = number of boundaries it ranks at or after;
 //   3. the groups' lists, each ascending by index, by per-thread chunk counts
 //      and one block scan per group; group k starts at c_{k-1}.
+// For N <= 40960 the order keys are first staged in shared memory, so the passes
+// do not wait on L2 latency for every element.
 #include "common.cuh"
 
 namespace hsa {
@@ -21,8 +25,13 @@ namespace hsa {
 constexpr int kSelectThreads = 1024;
 constexpr int kMaxGroups = 16;
 
+// Largest N whose keys are staged in shared memory (4 bytes each, on top of ~35 KB of
+// histograms); larger N reads the scores from global memory on every pass.
+constexpr int kSelectStagedMax = 40960;
+
 struct SelectArgs {
   int K;
+  int staged;               // 1: keys staged in dynamic shared memory
   int cum[kMaxGroups + 1];  // cum[0] = 0, cum[k] = n_1 + ... + n_k
 };
 
@@ -61,68 +70,147 @@ __device__ int block_exclusive_scan(int v, int* total, int* warp_sums) {
   return out;
 }
 
+// One radix pass over the keys that match `prefix` on `mask`: histogram of the 8-bit
+// digit at `shift` (per-warp private copies, then summed), and the digit holding the
+// element of rank `rank` among them.  Returns (digit, rank within that digit) through
+// shared memory.  Every thread of the block calls it.
+// Inverted order key of token n (ascending = descending score), from the keys staged in
+// shared memory when the kernel has them, else from the scores in global memory.
+struct KeySource {
+  const float* __restrict__ score;
+  const uint32_t* ikeys;  // shared memory, or nullptr
+  __device__ __forceinline__ uint32_t operator()(int n) const { return ikeys ? ikeys[n] : ~score_key(score[n]); }
+};
+
+__device__ void radix_pass(KeySource key, int N, uint32_t mask, uint32_t prefix, int shift,
+                           int rank, uint32_t (*hw)[257], uint32_t* hist, int* out_digit, int* out_rank) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = lane; i < 257; i += 32) hw[warp][i] = 0;
+  __syncwarp();
+  for (int n = tid; n < N; n += kSelectThreads) {
+    const uint32_t ik = key(n);
+    if ((ik & mask) == prefix) atomicAdd(&hw[warp][(ik >> shift) & 255u], 1u);
+  }
+  __syncthreads();
+  if (tid < 256) {
+    uint32_t t = 0;
+#pragma unroll 8
+    for (int w = 0; w < kSelectThreads / 32; ++w) t += hw[w][tid];
+    hist[tid] = t;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // lane l owns bins [8l, 8l+8): local sums, warp exclusive scan, then the lane whose
+    // range holds `rank` walks its 8 bins
+    uint32_t v[8], s = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      v[e] = hist[8 * lane + e];
+      s += v[e];
+    }
+    uint32_t incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t excl = incl - s;
+    if ((uint32_t)rank >= excl && (uint32_t)rank < incl) {
+      uint32_t r = (uint32_t)rank - excl;
+      int d = 0;
+      for (; d < 7; ++d) {
+        if (r < v[d]) break;
+        r -= v[d];
+      }
+      *out_digit = 8 * lane + d;
+      *out_rank = (int)r;
+    }
+  }
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kSelectThreads, 1)
     k_select(const float* __restrict__ score, int N, SelectArgs a, int8_t* __restrict__ group,
              int* __restrict__ order) {
+  __shared__ uint32_t hw[kSelectThreads / 32][257];   // per-warp private histograms
   __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist0[256];                      // first-pass histogram, shared by all boundaries
   __shared__ int warp_sums[33];
   __shared__ uint32_t s_thr_key[kMaxGroups];
   __shared__ int s_thr_idx[kMaxGroups];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_rank;
+  __shared__ int s_digit, s_rank;
+  extern __shared__ uint32_t s_ikeys[];                // N staged keys when the launch provides them
 
   const int tid = threadIdx.x;
   const int chunk = (N + kSelectThreads - 1) / kSelectThreads;
   const int lo = min(N, tid * chunk), hi = min(N, lo + chunk);
+  KeySource key{score, nullptr};
+  if (a.staged) {
+    for (int n = tid; n < N; n += kSelectThreads) s_ikeys[n] = ~score_key(score[n]);
+    __syncthreads();
+    key.ikeys = s_ikeys;
+  }
 
   // ---- 1. threshold element of every inner boundary
+  bool first_done = false;
   for (int b = 1; b < a.K; ++b) {
     const int c = a.cum[b];
     if (c <= 0 || c >= N) continue;  // empty prefix or everything: no threshold needed
-    // ascending order of ik = ~key is descending score order
+    // ascending order of ik = ~key is descending score order; find the element of rank c - 1
     uint32_t prefix = 0, mask = 0;
     int rank = c - 1;
     for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kSelectThreads) hist[i] = 0;
-      __syncthreads();
-      // warp-aggregated histogram: lanes with the same bin add once (scores share few
-      // exponent bytes, so plain per-lane atomics would serialise on one address)
-      const int lane = tid & 31;
-      for (int base = 0; base < N; base += kSelectThreads) {
-        const int n = base + tid;
-        uint32_t bin = 256u + (uint32_t)lane;          // unique non-bin value when inactive
-        if (n < N) {
-          const uint32_t ik = ~score_key(score[n]);
-          if ((ik & mask) == prefix) bin = (ik >> shift) & 255u;
+      if (shift == 24 && first_done) {
+        // the top-digit histogram does not depend on the boundary: reuse it
+        if (tid < 256) hist[tid] = hist0[tid];
+        __syncthreads();
+        if (tid < 32) {
+          uint32_t v[8], sum = 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            v[e] = hist[8 * tid + e];
+            sum += v[e];
+          }
+          uint32_t incl = sum;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (tid >= o) incl += y;
+          }
+          const uint32_t excl = incl - sum;
+          if ((uint32_t)rank >= excl && (uint32_t)rank < incl) {
+            uint32_t r = (uint32_t)rank - excl;
+            int d = 0;
+            for (; d < 7; ++d) {
+              if (r < v[d]) break;
+              r -= v[d];
+            }
+            s_digit = 8 * tid + d;
+            s_rank = (int)r;
+          }
         }
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-      }
-      __syncthreads();
-      if (tid == 0) {
-        int r = rank, d = 0;
-        for (; d < 255; ++d) {
-          if (r < (int)hist[d]) break;
-          r -= (int)hist[d];
+        __syncthreads();
+      } else {
+        radix_pass(key, N, mask, prefix, shift, rank, hw, hist, &s_digit, &s_rank);
+        if (shift == 24) {
+          if (tid < 256) hist0[tid] = hist[tid];
+          first_done = true;
         }
-        s_prefix = prefix | ((uint32_t)d << shift);
-        s_rank = r;
       }
-      __syncthreads();
-      prefix = s_prefix;
-      rank = s_rank;
+      prefix |= (uint32_t)s_digit << shift;
       mask |= 255u << shift;
+      rank = s_rank;
       __syncthreads();
     }
     // the rank-th smallest token index among keys equal to the target
     int cnt = 0;
-    for (int n = lo; n < hi; ++n) cnt += (~score_key(score[n]) == prefix);
+    for (int n = lo; n < hi; ++n) cnt += (key(n) == prefix);
     int total;
     const int excl = block_exclusive_scan(cnt, &total, warp_sums);
     if (rank >= excl && rank < excl + cnt) {
       int seen = excl;
       for (int n = lo; n < hi; ++n) {
-        if (~score_key(score[n]) == prefix) {
+        if (key(n) == prefix) {
           if (seen == rank) {
             s_thr_idx[b] = n;
             s_thr_key[b] = ~prefix;
@@ -140,7 +228,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
 #pragma unroll
   for (int k = 0; k < kMaxGroups; ++k) cnt[k] = 0;
   for (int n = lo; n < hi; ++n) {
-    const uint32_t key = score_key(score[n]);
+    const uint32_t kn = ~key(n);
     int g = 0;
     for (int b = 1; b < a.K; ++b) {
       const int c = a.cum[b];
@@ -148,7 +236,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
         ++g;
       } else if (c < N) {
         const uint32_t kt = s_thr_key[b];
-        if (key < kt || (key == kt && n > s_thr_idx[b])) ++g;
+        if (kn < kt || (kn == kt && n > s_thr_idx[b])) ++g;
       }
     }
     group[n] = (int8_t)g;
@@ -197,8 +285,19 @@ extern "C" int hsa_select_tokens(const float* d_score, int N, int K, const int* 
   }
   if (c != N) return set_error(HSA_EINVAL, "select: group sizes must sum to N");
   if (N == 0) return HSA_OK;
+  a.staged = N <= kSelectStagedMax ? 1 : 0;
+  const size_t dyn = a.staged ? (size_t)N * sizeof(uint32_t) : 0;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSelectStagedMax * (int)sizeof(uint32_t)) != cudaSuccess)
+      return check_launch("select: shared-memory attribute");
+    attr_done[dev] = true;
+  }
   ScopedTiming timing(HSA_KCLASS_OTHER, as_stream(stream));
-  k_select<<<1, kSelectThreads, 0, as_stream(stream)>>>(d_score, N, a, d_group, d_order);
+  k_select<<<1, kSelectThreads, dyn, as_stream(stream)>>>(d_score, N, a, d_group, d_order);
   count_launch(1);
   return check_launch("select launch");
 }
