@@ -223,35 +223,44 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
     __syncthreads();
   }
 
-  // ---- 2. group of each token in this thread's chunk; local counts per group
+  // ---- 2. group of each token in this thread's chunk; local counts per group.  Loops over
+  // groups are unrolled to kMaxGroups with a K guard, so cnt[] and off[] stay in registers.
   int cnt[kMaxGroups];
 #pragma unroll
   for (int k = 0; k < kMaxGroups; ++k) cnt[k] = 0;
   for (int n = lo; n < hi; ++n) {
     const uint32_t kn = ~key(n);
     int g = 0;
-    for (int b = 1; b < a.K; ++b) {
-      const int c = a.cum[b];
-      if (c <= 0) {
-        ++g;
-      } else if (c < N) {
-        const uint32_t kt = s_thr_key[b];
-        if (kn < kt || (kn == kt && n > s_thr_idx[b])) ++g;
+#pragma unroll
+    for (int b = 1; b < kMaxGroups; ++b) {
+      if (b < a.K) {
+        const int c = a.cum[b];
+        if (c <= 0) {
+          ++g;
+        } else if (c < N) {
+          const uint32_t kt = s_thr_key[b];
+          if (kn < kt || (kn == kt && n > s_thr_idx[b])) ++g;
+        }
       }
     }
     group[n] = (int8_t)g;
+    if (key.ikeys) s_ikeys[n] = (uint32_t)g;   // this thread's own slot: it now holds the group
 #pragma unroll
     for (int k = 0; k < kMaxGroups; ++k) cnt[k] += (g == k);
   }
 
   // ---- 3. ascending per-group lists, group k starting at cum[k]
   int off[kMaxGroups];
-  for (int k = 0; k < a.K; ++k) {
-    int total;
-    off[k] = a.cum[k] + block_exclusive_scan(cnt[k], &total, warp_sums);
+#pragma unroll
+  for (int k = 0; k < kMaxGroups; ++k) {
+    off[k] = 0;
+    if (k < a.K) {  // uniform over the block: every thread takes the same scans
+      int total;
+      off[k] = a.cum[k] + block_exclusive_scan(cnt[k], &total, warp_sums);
+    }
   }
   for (int n = lo; n < hi; ++n) {
-    const int g = group[n];
+    const int g = key.ikeys ? (int)s_ikeys[n] : (int)group[n];
 #pragma unroll
     for (int k = 0; k < kMaxGroups; ++k)
       if (k == g) order[off[k]++] = n;
