@@ -75,6 +75,31 @@ __device__ __forceinline__ float ex2_poly(float x) {
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
+// Packed fp32 pairs (two lanes of work per instruction on sm_100): d = a * b + c and d = a + b,
+// each component rounded like fmaf / __fadd_rn.
+__device__ __forceinline__ uint64_t as_u64(float2 v) {
+  return (uint64_t)__float_as_uint(v.x) | ((uint64_t)__float_as_uint(v.y) << 32);
+}
+__device__ __forceinline__ float2 as_f2(uint64_t v) {
+  return make_float2(__uint_as_float((uint32_t)v), __uint_as_float((uint32_t)(v >> 32)));
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(as_u64(a)), "l"(as_u64(b)), "l"(as_u64(c)));
+  return as_f2(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(as_u64(a)), "l"(as_u64(b)));
+  return as_f2(d);
+}
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -214,7 +239,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
 #pragma unroll
-      for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+      for (int c = 8; c < 64; c += 2)
+        mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
       const float mloc = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       // both halves of the row take the same max (double-buffered by tile parity)
@@ -248,19 +274,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       const float neg_m = -m;
+      const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(neg_m, neg_m);
       uint32_t pk[32];
-      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float2 rs4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        const float x0 = fmaf(__uint_as_float(sr[c]), sc, neg_m);
-        const float x1 = fmaf(__uint_as_float(sr[c + 1]), sc, neg_m);
+        const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
         const bool poly = (c & 7) >= 8 - kPolyPer8;  // compile-time per unrolled column pair
-        const float p0 = poly ? ex2_poly(x0) : ex2_approx(x0);
-        const float p1 = poly ? ex2_poly(x1) : ex2_approx(x1);
-        rs8[(c >> 1) & 7] += p0 + p1;
+        const float p0 = poly ? ex2_poly(x.x) : ex2_approx(x.x);
+        const float p1 = poly ? ex2_poly(x.y) : ex2_approx(x.y);
+        rs4[(c >> 1) & 3] = fadd2(rs4[(c >> 1) & 3], make_float2(p0, p1));
         pk[c >> 1] = pack_bf16x2(p0, p1);
       }
-      l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      l += ((rs4[0].x + rs4[0].y) + (rs4[1].x + rs4[1].y)) + ((rs4[2].x + rs4[2].y) + (rs4[3].x + rs4[3].y));
       // P buffer b was last read by PV_{j-2}
       if (j >= 2) mbar_wait(&sh->pv_done[b], ((j - 2) >> 1) & 1);
       __syncwarp();

@@ -87,9 +87,19 @@ __device__ void radix_pass(KeySource key, int N, uint32_t mask, uint32_t prefix,
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = lane; i < 257; i += 32) hw[warp][i] = 0;
   __syncwarp();
-  for (int n = tid; n < N; n += kSelectThreads) {
-    const uint32_t ik = key(n);
-    if ((ik & mask) == prefix) atomicAdd(&hw[warp][(ik >> shift) & 255u], 1u);
+  // Keys of similar scores share their top bytes, so most lanes of a warp often carry the
+  // same digit: the lanes equal to lane 0's digit add with one atomic, the rest one each.
+  for (int base = 0; base < N; base += kSelectThreads) {
+    const int n = base + tid;
+    uint32_t digit = 0xFFFFu;                       // no contribution
+    if (n < N) {
+      const uint32_t ik = key(n);
+      if ((ik & mask) == prefix) digit = (ik >> shift) & 255u;
+    }
+    const uint32_t lead = __shfl_sync(0xffffffffu, digit, 0);
+    const unsigned same = __ballot_sync(0xffffffffu, digit == lead);
+    if (lane == 0 && lead != 0xFFFFu) atomicAdd(&hw[warp][lead], (uint32_t)__popc(same));
+    if (digit != lead && digit != 0xFFFFu) atomicAdd(&hw[warp][digit], 1u);
   }
   __syncthreads();
   if (tid < 256) {

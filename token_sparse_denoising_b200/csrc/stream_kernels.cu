@@ -11,6 +11,8 @@
 //
 // All rows are read and written with 16-byte vectors; one warp owns one row,
 // so a row's reduction stays in registers and warp shuffles.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace hsa {
@@ -37,6 +39,13 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
   return make_float4(fa.x, fa.y, fb.x, fb.y);
 }
 __device__ __forceinline__ void store4(float* p, float4 v) { st4(p, v); }
+// raw register forms of 4 consecutive elements, widened to float
+__device__ __forceinline__ float4 widen4(float4 v) { return v; }
+__device__ __forceinline__ float4 widen4(uint2 u) {
+  const float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
+  const float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
+  return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
 __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
   __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
   uint2 u;
@@ -272,8 +281,14 @@ __device__ __forceinline__ float2 rope_cs(int c, int pf, int ph, int pw) {
   const float p = (float)(axis == 0 ? pf : (axis == 1 ? ph : pw));
   // 10000^(-2j/w) = 2^(-(2j/w) * log2(10000))
   const float inv_freq = exp2f(-(float)(2 * j) / (float)w * 13.287712379549449f);
+  // angle reduced to [-pi, pi] by k multiples of 2 pi, 2 pi split into a float head and its
+  // remainder (Cody-Waite), then the fast intrinsic; angles here are position x frequency,
+  // below ~100 rad, so the reduction error stays near 1e-6
+  const float ang = p * inv_freq;
+  const float k = rintf(ang * 0.15915494309189535f);
+  const float r = fmaf(-k, -1.7484556025237907e-07f, fmaf(-k, 6.2831854820251465f, ang));
   float sn, cs;
-  sincosf(p * inv_freq, &sn, &cs);
+  __sincosf(r, &sn, &cs);
   return make_float2(cs, sn);
 }
 
@@ -297,15 +312,21 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope(const TIn* __restrict__ qk
   }
   const int pf = pos[3 * n + 0], ph = pos[3 * n + 1], pw = pos[3 * n + 2];
   const TIn* row = qkv + (size_t)r * 3 * D;
-  float4 q[VPT], k[VPT];
+  // q and k stay in registers in their input type (bf16: 8 bytes per 4 channels) and v is
+  // copied to the cache in this first pass, so the second pass holds only q, k and the
+  // gains: 128 registers instead of 189 for D = 1536, two CTAs per SM instead of one
+  using Raw = typename std::conditional<sizeof(TIn) == 2, uint2, float4>::type;
+  Raw q[VPT], k[VPT];
   float sq = 0.f, sk = 0.f;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int c = (i * 32 + lane) * 4;
-    q[i] = load4(row + c);
-    k[i] = load4(row + D + c);
-    sq += q[i].x * q[i].x + q[i].y * q[i].y + q[i].z * q[i].z + q[i].w * q[i].w;
-    sk += k[i].x * k[i].x + k[i].y * k[i].y + k[i].z * k[i].z + k[i].w * k[i].w;
+    q[i] = *reinterpret_cast<const Raw*>(row + c);
+    k[i] = *reinterpret_cast<const Raw*>(row + D + c);
+    store4(Vc + (size_t)n * D + c, load4(row + 2 * D + c));
+    const float4 a = widen4(q[i]), b = widen4(k[i]);
+    sq += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+    sk += b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
   }
   const float rq = rsqrtf(warp_sum(sq) * (1.0f / D) + kNormEps);
   const float rk = rsqrtf(warp_sum(sk) * (1.0f / D) + kNormEps);
@@ -314,8 +335,9 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope(const TIn* __restrict__ qk
     const int c = (i * 32 + lane) * 4;
     const int ch = c & 127;  // channel within the head; c..c+3 stay in one head
     const float4 gq = ld4(g_q + c), gk = ld4(g_k + c);
-    const float4 a = make_float4(q[i].x * rq * gq.x, q[i].y * rq * gq.y, q[i].z * rq * gq.z, q[i].w * rq * gq.w);
-    const float4 b = make_float4(k[i].x * rk * gk.x, k[i].y * rk * gk.y, k[i].z * rk * gk.z, k[i].w * rk * gk.w);
+    const float4 qv = widen4(q[i]), kv = widen4(k[i]);
+    const float4 a = make_float4(qv.x * rq * gq.x, qv.y * rq * gq.y, qv.z * rq * gq.z, qv.w * rq * gq.w);
+    const float4 b = make_float4(kv.x * rk * gk.x, kv.y * rk * gk.y, kv.z * rk * gk.z, kv.w * rk * gk.w);
     const float2 t0 = rope_cs(ch, pf, ph, pw), t1 = rope_cs(ch + 2, pf, ph, pw);
     float4 qo, ko;
     qo.x = a.x * t0.x - a.y * t0.y;  qo.y = a.x * t0.y + a.y * t0.x;
@@ -324,7 +346,6 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope(const TIn* __restrict__ qk
     ko.z = b.z * t1.x - b.w * t1.y;  ko.w = b.z * t1.y + b.w * t1.x;
     store4(Q + (size_t)r * D + c, qo);
     store4(Kc + (size_t)n * D + c, ko);
-    store4(Vc + (size_t)n * D + c, load4(row + 2 * D + c));
   }
 }
 
