@@ -7,20 +7,28 @@
 //   K, V: L x 128H cache rows, o: M x 128H.  Non-causal.
 //
 // One CTA = one head x 128 queries, streaming 128-key tiles of K and V.
-//   warp 0      TMA producer: Q once; K_j into a 3-slot ring, V_j into a 2-slot ring
-//   warp 1      TMEM owner (512 columns) and MMA issuer:
-//                 S_j = Q K_j^T        (SS: both K-major, 128 x 128 x 128)
-//                 O  += P_j V_j        (TS: P from TMEM, V MN-major)
-//               S_{j+1} is issued before waiting for P_j, so QK^T of the next
-//               tile overlaps the softmax of this one.
-//   warps 2..9  softmax: two threads per query row, each owning 64 of the 128 key
-//               columns of a tile (warps 2-5 the left half, 6-9 the right half;
-//               warp w reads TMEM lane quarter w % 4).  The two halves of a row
-//               agree on the row max through shared memory and a named barrier per
-//               lane quarter.  p = 2^(t - m) goes back to TMEM as bf16.  O is
-//               rescaled in TMEM only when the max grew by more than 2^8
-//               (otherwise the stale max keeps p <= 256, safe in fp32).
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
+//   warp 0      TMA producer (the warp waits, one elected lane copies): Q once; K_j into a 3-slot ring, V_j into a 2-slot ring,
+//               in the order the MMA warp consumes them (K0 K1 V0 K2 V1 K3 ...)
+//   warp 1      TMEM owner (512 columns) and MMA issuer (the warp runs the loop with
+//               warp-uniform descriptors, one elected lane issues):
+//                 S_b = Q K_j^T          (SS: both K-major, 128 x 128 x 128), b = j % 2
+//                 O_b += P_j V_j         (TS: P from TMEM, V MN-major)
+//               QK^T of tile j+2 is issued right after PV of tile j, so the tensor
+//               pipe alternates between the two parities.
+//   warps 2..9  softmax, one thread per query row and all 128 key columns of a tile:
+//               warps 2-5 take the even tiles, warps 6-9 the odd tiles (warp w reads
+//               TMEM lane quarter w % 4).  Each parity keeps its own running max, sum
+//               and O accumulator, so the two warps of a sub-partition never wait for
+//               each other and one's exponentials overlap the other's loads, max and
+//               stores.  p = 2^(t - m) goes back to TMEM as bf16 over the first 64
+//               columns of the S buffer it came from.  O_b is rescaled in TMEM only
+//               when the max grew by more than 2^8 (the stale max keeps p <= 256).
+//               The epilogue merges the two parities: O = (a0 O_0 + a1 O_1) / (a0 l_0
+//               + a1 l_1) with a_b = 2^(m_b - max(m_0, m_1)).
+// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_b aliases the
+// first 64 columns of S_b.  QK^T of tile j+2 overwrites S_b only after PV of tile j
+// has read P_b: both are issued by the one MMA thread, whose tcgen05.mma operations
+// execute in issue order.
 // Key rows beyond L are zero-filled by TMA and masked to -inf; query rows beyond
 // M are computed on zeros and never stored.
 #include "tcgen05.cuh"
@@ -33,9 +41,9 @@ constexpr int kKSlots = 3;
 constexpr int kVSlots = 2;
 constexpr int kAttnThreads = 320;                 // 2 control warps + 8 softmax warps
 constexpr int kTileBytes = 128 * 128 * 2;         // one 128 x 128 bf16 operand tile (two 64-column boxes)
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+constexpr uint32_t kColS = 0, kColO = 256;
 // Exponentials computed with the polynomial instead of the MUFU unit: the columns c
-// of a thread's 64 with (c % 8) >= 8 - kPolyPer8.  Measured at the Wan-1.3B shape
+// of a thread's 128 with (c % 8) >= 8 - kPolyPer8.  Measured at the Wan-1.3B shape
 // (attention alone, 32760 x 32760, 12 heads): 0 of 8 -> 6.44 ms, 2 of 8 -> 7.04 ms,
 // 4 of 8 -> 7.63 ms, so the MUFU path alone is the default.
 #ifndef HSA_ATTN_POLY_PER8
@@ -47,10 +55,9 @@ struct AttnShared {
   uint64_t q_full;
   uint64_t k_full[kKSlots], k_empty[kKSlots];
   uint64_t v_full[kVSlots], v_empty[kVSlots];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t s_full[2], p_full[2], o_done;
   uint32_t tmem;
-  float xmax[2][2][128];  // [tile parity][column half][row]: row-max exchange
-  float xsum[2][128];     // [column half][row]: final row-sum exchange
+  float xm[2][128], xl[2][128];  // [parity][row]: running max and sum, merged in the epilogue
 };
 constexpr int kAttnSmem = kTileBytes * (1 + kKSlots + kVSlots) + 1024 + (int)sizeof(AttnShared);
 
@@ -130,10 +137,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->s_full[b], 1);
-      mbar_init(&sh->s_free[b], 256);
-      mbar_init(&sh->p_full[b], 256);
-      mbar_init(&sh->pv_done[b], 1);
+      mbar_init(&sh->p_full[b], 128);
     }
+    mbar_init(&sh->o_done, 1);
     fence_mbar_init();
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
@@ -149,176 +155,220 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tm = sh->tmem;
 
   if (warp == 0) {
-    if (lane == 0) {
-      const int x0 = h * 128;
+    // TMA producer: the whole warp runs the loop and waits; one elected lane issues the copies
+    const int x0 = h * 128;
+    const bool leader = elect_one();
+    if (leader) {
       mbar_expect_tx(&sh->q_full, kTileBytes);
       tma_load_2d(sQ, &tmQ, &sh->q_full, x0, m0);
       tma_load_2d(sQ + kTileBytes / 2, &tmQ, &sh->q_full, x0 + 64, m0);
-      for (int j = 0; j < nj; ++j) {
-        const int sk = j % kKSlots, sv = j % kVSlots;
-        if (!mbar_wait(&sh->k_empty[sk], ((j / kKSlots) & 1) ^ 1)) break;
+    }
+    auto load_k = [&](int j) -> bool {
+      const int sk = j % kKSlots;
+      const bool ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->k_empty[sk], ((j / kKSlots) & 1) ^ 1), 0);
+      __syncwarp();
+      if (ok && leader) {
         uint8_t* k = sK + sk * kTileBytes;
         mbar_expect_tx(&sh->k_full[sk], kTileBytes);
         tma_load_2d(k, &tmK, &sh->k_full[sk], x0, j * kAttnBN);
         tma_load_2d(k + kTileBytes / 2, &tmK, &sh->k_full[sk], x0 + 64, j * kAttnBN);
-        if (!mbar_wait(&sh->v_empty[sv], ((j / kVSlots) & 1) ^ 1)) break;
+      }
+      return ok;
+    };
+    bool ok = load_k(0);
+    if (ok && nj > 1) ok = load_k(1);
+    for (int j = 0; ok && j < nj; ++j) {
+      const int sv = j % kVSlots;
+      ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->v_empty[sv], ((j / kVSlots) & 1) ^ 1), 0);
+      __syncwarp();
+      if (!ok) break;
+      if (leader) {
         uint8_t* v = sV + sv * kTileBytes;
         mbar_expect_tx(&sh->v_full[sv], kTileBytes);
         tma_load_2d(v, &tmV, &sh->v_full[sv], x0, j * kAttnBN);
         tma_load_2d(v + kTileBytes / 2, &tmV, &sh->v_full[sv], x0 + 64, j * kAttnBN);
       }
+      if (j + 2 < nj) ok = load_k(j + 2);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
-      const uint32_t q_addr = smem_u32(sQ);
-      bool ok = mbar_wait(&sh->q_full, 0);
-      auto issue_qk = [&](int j) -> bool {
-        const int sk = j % kKSlots, b = j & 1;
-        if (!mbar_wait(&sh->k_full[sk], (j / kKSlots) & 1)) return false;
-        if (j >= 2 && !mbar_wait(&sh->s_free[b], ((j - 2) >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + sk * kTileBytes);
+    // MMA issuer: the whole warp runs the loop, waits and builds the descriptors (warp-uniform
+    // values); one elected lane issues each tcgen05.mma and commit
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
+    const bool leader = elect_one();
+    // descriptor of a shared-memory address a: desc(base) + (a - base) / 16 (the start-address
+    // field is the low 14 bits of a / 16 and never carries: shared memory is below 256 KB)
+    const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t k_desc = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t v_desc = sdesc_sw128(smem_u32(sV), kTileBytes / 2, 1024);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      const bool r = __shfl_sync(0xffffffffu, mbar_wait(bar, parity), 0);
+      __syncwarp();
+      return r;
+    };
+    auto issue_qk = [&](int j) -> bool {
+      const int sk = j % kKSlots, b = j & 1;
+      if (!wait_all(&sh->k_full[sk], (j / kKSlots) & 1)) return false;
+      tc_fence_after();
+      const uint64_t kd = k_desc + (uint64_t)((sk * kTileBytes) >> 4);
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-          umma_ss(tm + kColS + b * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
-                  idesc_s, kk > 0);
+          const uint32_t off = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
+          umma_ss(tm + kColS + b * 128, q_desc + off, kd + off, idesc_s, kk > 0);
         }
         umma_commit(&sh->s_full[b]);
-        umma_commit(&sh->k_empty[sk]);          // K_j is free once S_j is computed
-        return true;
-      };
-      if (ok) ok = issue_qk(0);
-      for (int j = 0; ok && j < nj; ++j) {
-        if (j + 1 < nj && !issue_qk(j + 1)) break;
-        const int b = j & 1, sv = j % kVSlots;
-        if (!mbar_wait(&sh->p_full[b], (j >> 1) & 1)) break;
-        if (!mbar_wait(&sh->v_full[sv], (j / kVSlots) & 1)) break;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sV + sv * kTileBytes);
+        umma_commit(&sh->k_empty[sk]);        // K_j is free once S_j is computed
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = wait_all(&sh->q_full, 0);
+    if (ok) ok = issue_qk(0);
+    if (ok && nj > 1) ok = issue_qk(1);
+    for (int j = 0; ok && j < nj; ++j) {
+      const int b = j & 1, sv = j % kVSlots;
+      if (!wait_all(&sh->p_full[b], (j >> 1) & 1)) break;
+      if (!wait_all(&sh->v_full[sv], (j / kVSlots) & 1)) break;
+      tc_fence_after();
+      const uint64_t vd = v_desc + (uint64_t)((sv * kTileBytes) >> 4);
+      if (leader) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // V tile: key rows of 128 B (64 channels) per box; 16 keys = two 1024-byte atoms
-          umma_ts(tm + kColO, tm + kColP + b * 64 + kk * 8, sdesc_sw128(v_addr + kk * 2048, kTileBytes / 2, 1024),
-                  idesc_o, (j > 0 || kk > 0));
+          umma_ts(tm + kColO + b * 128, tm + kColS + b * 128 + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), idesc_o,
+                  (j >= 2 || kk > 0));
         }
-        umma_commit(&sh->pv_done[b]);
         umma_commit(&sh->v_empty[sv]);
       }
+      __syncwarp();
+      if (j + 2 < nj) ok = issue_qk(j + 2);   // overwrites S_b (P_j) after PV_j in issue order
     }
+    if (leader) umma_commit(&sh->o_done);   // every MMA of this CTA, both O accumulators
+    __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax warps
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;               // key-column half of the tile this thread owns
+    const int par = (warp - 2) >> 2;                // tile parity this warp handles
     const int row = quarter * 32 + lane;
-    const int bar_id = 1 + quarter;                 // named barrier of the two warps of this quarter
     const uint32_t lane_base = tm + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t s_col = lane_base + kColS + par * 128, o_col = lane_base + kColO + par * 128;
     const float sc = 0.12751743074680484f;          // log2(e) / sqrt(128)
     float m = -INFINITY, l = 0.f;
-    for (int j = 0; j < nj; ++j) {
-      const int b = j & 1;
-      mbar_wait(&sh->s_full[b], (j >> 1) & 1);
+    for (int j = par; j < nj; j += 2) {
+      mbar_wait(&sh->s_full[par], (j >> 1) & 1);
       __syncwarp();
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(lane_base + kColS + b * 128 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(sr));
-      tmem_ld32(lane_base + kColS + b * 128 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+      uint32_t sr[128];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+        tmem_ld32(s_col + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + q4 * 32));
       tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&sh->s_free[b]);
 
       if ((j + 1) * kAttnBN > L) {  // ragged last tile only: keys beyond L get -inf
-        const int valid = L - j * kAttnBN - half * 64;
+        const int valid = L - j * kAttnBN;
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < 128; ++c)
           if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
       }
       float mx8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
 #pragma unroll
-      for (int c = 8; c < 64; c += 2)
+      for (int c = 8; c < 128; c += 2)
         mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-      const float mloc = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      // both halves of the row take the same max (double-buffered by tile parity)
-      sh->xmax[b][half][row] = mloc;
-      named_bar_sync(bar_id, 64);
-      const float m_tile = sc * fmaxf(mloc, sh->xmax[b][half ^ 1][row]);
-      if (j == 0) {
+      const float m_tile = sc * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                      fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      // lazy rescale: the max moves only when it grew by more than 2^8; O_par is then scaled
+      // after P is stored, when the S registers are free
+      bool need = false;
+      float corr = 1.0f;
+      if (j == par) {
         m = m_tile;
-      } else {
-        const bool need = m_tile > m + 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          // O must hold PV_{j-1} before it is rescaled; each half rescales its 64 columns of O
-          mbar_wait(&sh->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1);
-          __syncwarp();
-          tc_fence_after();
-          const float corr = need ? ex2_approx(m - m_tile) : 1.0f;
-#pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + kColO + half * 64 + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-            tmem_st32(lane_base + kColO + half * 64 + c * 32, o);
-          }
-          tmem_st_wait();
-          if (need) {
-            l *= corr;
-            m = m_tile;
-          }
-        }
+      } else if (m_tile > m + 8.0f) {
+        need = true;
+        corr = ex2_approx(m - m_tile);
+        l *= corr;
+        m = m_tile;
       }
       const float neg_m = -m;
       const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(neg_m, neg_m);
-      uint32_t pk[32];
       float2 rs4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
-        const bool poly = (c & 7) >= 8 - kPolyPer8;  // compile-time per unrolled column pair
-        const float p0 = poly ? ex2_poly(x.x) : ex2_approx(x.x);
-        const float p1 = poly ? ex2_poly(x.y) : ex2_approx(x.y);
-        rs4[(c >> 1) & 3] = fadd2(rs4[(c >> 1) & 3], make_float2(p0, p1));
-        pk[c >> 1] = pack_bf16x2(p0, p1);
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = hh * 64; c < hh * 64 + 64; c += 2) {
+          const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
+          const bool poly = (c & 7) >= 8 - kPolyPer8;  // compile-time per unrolled column pair
+          const float p0 = poly ? ex2_poly(x.x) : ex2_approx(x.x);
+          const float p1 = poly ? ex2_poly(x.y) : ex2_approx(x.y);
+          rs4[(c >> 1) & 3] = fadd2(rs4[(c >> 1) & 3], make_float2(p0, p1));
+          pk[(c >> 1) & 31] = pack_bf16x2(p0, p1);
+        }
+        // P column i holds keys 2i, 2i+1 of the tile, over S_par's first 64 columns
+        tmem_st32(s_col + hh * 32, pk);
       }
       l += ((rs4[0].x + rs4[0].y) + (rs4[1].x + rs4[1].y)) + ((rs4[2].x + rs4[2].y) + (rs4[3].x + rs4[3].y));
-      // P buffer b was last read by PV_{j-2}
-      if (j >= 2) mbar_wait(&sh->pv_done[b], ((j - 2) >> 1) & 1);
-      __syncwarp();
-      tc_fence_after();
-      tmem_st32(lane_base + kColP + b * 64 + half * 32, pk);
+      if (__any_sync(0xffffffffu, need)) {
+        // O_par holds PV of this parity's previous tile, complete: S_par was written by an MMA
+        // issued after that PV, and the s_full wait above covered it.  PV of this tile starts
+        // only after the p_full arrival below.
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_col + c * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+          tmem_st32(o_col + c * 32, o);
+        }
+      }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&sh->p_full[b]);
+      mbar_arrive(&sh->p_full[par]);
     }
     // ---------------------------------------------------------------- epilogue
-    sh->xsum[half][row] = l;
-    named_bar_sync(bar_id, 64);
-    const float inv_l = 1.0f / (l + sh->xsum[half ^ 1][row]);
-    mbar_wait(&sh->pv_done[(nj - 1) & 1], ((nj - 1) >> 1) & 1);
+    // merge the two parities; parity 1 has tiles only when nj >= 2
+    sh->xm[par][row] = m;
+    sh->xl[par][row] = l;
+    named_bar_sync(1 + quarter, 64);                // the even and the odd warp of this lane quarter
+    const bool two = nj >= 2;
+    const float m0v = sh->xm[0][row], m1v = sh->xm[1][row];
+    const float mm = two ? fmaxf(m0v, m1v) : m0v;
+    const float a0 = ex2_approx(m0v - mm);
+    const float a1 = two ? ex2_approx(m1v - mm) : 0.f;
+    const float inv_l = 1.0f / (a0 * sh->xl[0][row] + a1 * sh->xl[1][row]);
+    const float w0 = a0 * inv_l, w1 = a1 * inv_l;
+    mbar_wait(&sh->o_done, 0);
     __syncwarp();
     tc_fence_after();
     const int grow = m0 + row;
+    // this warp writes output columns [par * 64, par * 64 + 64) of the head
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
-      uint32_t o[32];
-      __syncwarp();  // reconverge after the guarded stores before the warp-collective load
-      tmem_ld32(lane_base + kColO + half * 64 + c * 32, o);
+      const uint32_t col = (uint32_t)(par * 64 + c * 32);
+      uint32_t o0[32], o1[32];
+      __syncwarp();  // reconverge after the guarded stores before the warp-collective loads
+      tmem_ld32(lane_base + kColO + col, o0);
+      if (two) tmem_ld32(lane_base + kColO + 128 + col, o1);
       tmem_ld_wait();
+      if (!two) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o1[e] = 0u;
+      }
       if (grow < M) {
-        __nv_bfloat16* dst = O + (size_t)grow * (H * 128) + h * 128 + half * 64 + c * 32;
+        __nv_bfloat16* dst = O + (size_t)grow * (H * 128) + h * 128 + col;
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
+          float f[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) f[t] = fmaf(__uint_as_float(o0[e + t]), w0, __uint_as_float(o1[e + t]) * w1);
           uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
-          u.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
-          u.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
-          u.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+          u.x = pack_bf16x2(f[0], f[1]);
+          u.y = pack_bf16x2(f[2], f[3]);
+          u.z = pack_bf16x2(f[4], f[5]);
+          u.w = pack_bf16x2(f[6], f[7]);
           *reinterpret_cast<uint4*>(dst + e) = u;
         }
       }
