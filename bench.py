@@ -337,7 +337,8 @@ def run_gpu(args, rank, world, barrier, allmax):
 
 def run_loop(args):
     """Full Wan-1.3B-shaped loop: latent 16x21x60x104 patchified 1x2x2 (N=32760, C=64), 30 blocks,
-    T=40; HSA with budgets {40,20,10} sized 25/25/50 % and m=4 against the uniform 40-step run."""
+    T=40; HSA with budgets {40,20,10} sized 25/25/50 % and m=4 against the uniform 40-step run.
+    Each run is timed eagerly (host launches) and as one recorded CUDA graph of all T steps."""
     import torch
     from token_sparse_denoising_b200 import hsa, pipeline
     hsa.load()
@@ -363,7 +364,27 @@ def run_loop(args):
         assert hsa.device_status() == 0
         out[name] = {"ms": round(a.elapsed_time(b), 1), "token_steps": int(run.n_active.sum()),
                      "active_fraction": round(float(run.n_active.sum()) / (wl.T * N), 4)}
+        x_eager = run.x.clone()
+        # the same run recorded as one CUDA graph (every launch of all T steps) and replayed
+        run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift)
+        n0 = hsa.launch_count()
+        t0 = time.perf_counter()
+        g = run.capture()
+        torch.cuda.synchronize()
+        cap_s = time.perf_counter() - t0
+        recorded = hsa.launch_count() - n0
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        run.replay(g)
+        b.record()
+        b.synchronize()
+        assert hsa.device_status() == 0
+        out[name]["graph"] = {"ms": round(a.elapsed_time(b), 1), "capture_s": round(cap_s, 2),
+                              "launches_recorded": int(recorded),
+                              "bitwise_equal_to_eager": bool(torch.equal(run.x, x_eager))}
+        del g
     out["speedup"] = round(out["uniform"]["ms"] / out["hsa"]["ms"], 3)
+    out["speedup_graph"] = round(out["uniform"]["graph"]["ms"] / out["hsa"]["graph"]["ms"], 3)
     return out
 
 

@@ -166,13 +166,20 @@ def l1_score(v_new, v_prev, score, stream=None):
     _check(lib().hsa_l1_score(_ptr(v_new), _ptr(v_prev), N, Cc, _ptr(score), _stream(stream)), "hsa_l1_score")
 
 
-def select_tokens(score, group_sizes, group, order, stream=None):
+def select_tokens_workspace_size(N: int, K: int) -> int:
+    return int(lib().hsa_select_tokens_workspace_size(N, K))
+
+
+def select_tokens(score, group_sizes, group, order, stream=None, ws=None):
     import torch
     N = score.shape[0]
     K = len(group_sizes)
     sizes = np.ascontiguousarray(group_sizes, np.int32)
     nbytes = lib().hsa_select_tokens_workspace_size(N, K)
-    ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=score.device)
+    if ws is None:
+        ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=score.device)
+    elif ws.numel() * ws.element_size() < nbytes:
+        raise ValueError("select_tokens: workspace smaller than hsa_select_tokens_workspace_size")
     _check(lib().hsa_select_tokens(_ptr(score), N, K, sizes.ctypes.data, _ptr(group), _ptr(order), _ptr(ws),
                                    nbytes, _stream(stream)), "hsa_select_tokens")
 

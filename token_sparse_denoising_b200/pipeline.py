@@ -118,8 +118,38 @@ class HSARun:
         self.group = torch.zeros(N, dtype=torch.int8, device=device)
         self.score = torch.zeros(N, dtype=torch.float32, device=device)
         self.idx_buf = torch.empty(N, dtype=torch.int32, device=device)
+        self.sel_ws = torch.empty(max(hsa.select_tokens_workspace_size(N, len(self.sizes)), 1), dtype=torch.uint8,
+                                  device=device)
         self.starts = np.concatenate([[0], np.cumsum(self.sizes)]).astype(np.int64)
         self.i = 0
+
+    def reset(self, x0, vhat0):
+        """Start the run again from (x0, vhat0) in the same device buffers, so a captured graph of
+        the loop can be replayed for a new latent."""
+        self.x.copy_(torch.as_tensor(np.ascontiguousarray(x0, np.float32)))
+        self.vhat.copy_(torch.as_tensor(np.ascontiguousarray(vhat0, np.float32)))
+        self.order.copy_(torch.arange(self.N, dtype=torch.int32))
+        self.group.zero_()
+        self.score.zero_()
+        self.i = 0
+
+    def capture(self):
+        """Record the remaining steps of the run (every launch of every step, selection included)
+        as one CUDA graph and return it; replaying it runs those steps.  The schedule is fixed on
+        the host, and the active index lists live at fixed device addresses whose contents the
+        selection kernel rewrites, so one recording serves every replay.  Nothing executes
+        during the recording: the state stays where it was, and replay(g) then runs the steps."""
+        g = torch.cuda.CUDAGraph()
+        i0 = self.i
+        with torch.cuda.graph(g):
+            self.run()
+        self.i = i0
+        return g
+
+    def replay(self, g):
+        """Run a graph from capture() on the current state (reset() first for a new latent)."""
+        g.replay()
+        self.i = self.T
 
     def active_index(self, i: int):
         act = self.table[i].astype(bool)
@@ -144,7 +174,7 @@ class HSARun:
         dsig = float(np.float32(self.sigmas[i + 1]) - np.float32(self.sigmas[i]))
         hsa.euler_update(self.x, self.vhat, vA, idx, dsig, score=self.score if full else None)
         if full:
-            hsa.select_tokens(self.score, self.sizes, self.group, self.order)
+            hsa.select_tokens(self.score, self.sizes, self.group, self.order, ws=self.sel_ws)
         if record is not None:
             record.append({"i": i, "M": int(idx.shape[0]), "full": full,
                            "score": self.score.cpu().numpy().copy() if full else None,
