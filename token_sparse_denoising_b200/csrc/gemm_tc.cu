@@ -11,9 +11,11 @@
 //               issues tcgen05.mma (M=128, N=BN, K=16) into the free one and
 //               releases each shared-memory slot with tcgen05.commit;
 //   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter, bias, GELU /
-//               residual gate.  Thread = output row.  bf16 outputs are staged per
-//               warp as 32 x 32 sub-tiles in shared memory and written by TMA stores;
-//               the fp32 residual update reads and writes rows directly.
+//               residual gate.  Thread = output row.  Each warp stages 32 x 32
+//               sub-tiles of the output in shared memory and hands them to the TMA:
+//               bf16 and fp32 outputs by tensor stores, the fp32 residual update
+//               y += gate * (acc + b) by a tensor reduce-add done in L2, so the
+//               epilogue never waits on a global load.
 // Rows beyond M are zero-filled by TMA and never stored.
 #include "tcgen05.cuh"
 
@@ -31,60 +33,16 @@ struct GemmCfg {
   static constexpr int kABytes = kGemmBM * kGemmBK * 2;   // 16 KB
   static constexpr int kBBytes = BN * kGemmBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  // epilogue staging for the bf16 outputs: 4 warps x 2 buffers x (32 rows x 64 bytes)
-  static constexpr int kStageOutBytes = 4 * 2 * 2048;
+  // epilogue staging: 4 warps x 2 buffers x one 32 x 32 sub-tile (fp32: 4 KB; bf16 uses 2 KB of it)
+  static constexpr int kStageOutBytes = 4 * 2 * 4096;
   static constexpr int kSmem = kStages * kStageBytes + kStageOutBytes + 1024 /*align*/ + 256 /*barriers*/;
   static_assert(2 * BN <= 512, "double-buffered accumulator must fit TMEM");
+  static_assert(kSmem <= 232448, "GEMM shared memory above the 227 KB per-CTA limit");
 };
 
 __device__ __forceinline__ float gelu_tanh_f(float x) {
   const float u = 0.7978845608028654f * (x + 0.044715f * x * x * x);
   return 0.5f * x * (1.0f + tanhf(u));
-}
-
-// Epilogue of 32 accumulator columns of one output row (thread = row).
-template <int EPI>
-__device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row, int col0, int Nout,
-                                               const float* __restrict__ bias, const float* __restrict__ gate,
-                                               void* __restrict__ out) {
-  float v[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + (bias ? __ldg(bias + col0 + j) : 0.f);
-  if constexpr (EPI == EPI_STORE || EPI == EPI_GELU) {
-    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * Nout + col0;
-#pragma unroll
-    for (int j = 0; j < 32; j += 8) {
-      float t[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) t[e] = EPI == EPI_GELU ? gelu_tanh_f(v[j + e]) : v[j + e];
-      uint4 u;
-      u.x = pack_bf16x2(t[0], t[1]);
-      u.y = pack_bf16x2(t[2], t[3]);
-      u.z = pack_bf16x2(t[4], t[5]);
-      u.w = pack_bf16x2(t[6], t[7]);
-      *reinterpret_cast<uint4*>(y + j) = u;
-    }
-  } else if constexpr (EPI == EPI_F32) {
-    float* y = reinterpret_cast<float*>(out) + (size_t)row * Nout + col0;
-#pragma unroll
-    for (int j = 0; j < 32; j += 4)
-      *reinterpret_cast<float4*>(y + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-  } else {  // EPI_RESID: y += gate * (acc + b)
-    float* y = reinterpret_cast<float*>(out) + (size_t)row * Nout + col0;
-    float4 o[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) o[j] = *reinterpret_cast<const float4*>(y + 4 * j);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (gate) g = __ldg(reinterpret_cast<const float4*>(gate + col0 + 4 * j));
-      o[j].x = fmaf(g.x, v[4 * j + 0], o[j].x);
-      o[j].y = fmaf(g.y, v[4 * j + 1], o[j].y);
-      o[j].z = fmaf(g.z, v[4 * j + 2], o[j].z);
-      o[j].w = fmaf(g.w, v[4 * j + 3], o[j].w);
-      *reinterpret_cast<float4*>(y + 4 * j) = o[j];
-    }
-  }
 }
 
 // Persistent: CTA c handles output tiles c, c + gridDim.x, ... (n fastest, so the
@@ -98,7 +56,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const float* __restrict__ gate, void* __restrict__ out) {
   using Cfg = GemmCfg<BN>;
   constexpr int S = Cfg::kStages;
-  constexpr bool kTmaOut = (EPI == EPI_STORE || EPI == EPI_GELU);
+  constexpr bool kF32Out = (EPI == EPI_RESID || EPI == EPI_F32);
+  constexpr int kChunkBytes = kF32Out ? 4096 : 2048;   // one staged 32 x 32 output sub-tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_out = smem + S * Cfg::kStageBytes;   // 1024-aligned
@@ -125,7 +84,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    if (kTmaOut) prefetch_tmap(&tmY);
+    prefetch_tmap(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 2 * BN);
@@ -181,12 +140,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows of that quarter
     const int quarter = warp & 3;
-    uint8_t* my_out = stage_out + (warp - 2) * 2 * 2048;   // this warp's two 32 x 32 bf16 buffers
+    uint8_t* my_out = stage_out + (warp - 2) * 2 * kChunkBytes;   // this warp's two sub-tile buffers
     int tc = 0, nchunk = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
       const int n0 = (t % n_tiles) * BN, m0 = (t / n_tiles) * kGemmBM;
       const int buf = tc & 1;
-      const int row = m0 + quarter * 32 + lane;
       const bool ok = mbar_wait(&acc_full[buf], (tc >> 1) & 1);
       __syncwarp();
       tc_fence_after();
@@ -201,14 +159,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_before();
           mbar_arrive(&acc_empty[buf]);
         }
-        if constexpr (kTmaOut) {
-          // stage the warp's 32 x 32 sub-tile (64-byte swizzle: chunk k of row r at k ^ ((r>>1)&3),
-          // conflict-free for thread-per-row writes) and store it with one TMA copy; rows
-          // beyond M are clipped by the tensor map
-          uint8_t* sb = my_out + (nchunk & 1) * 2048;
-          if (lane == 0) bulk_wait_group_read<1>();   // the store that last read sb is done
-          __syncwarp();
-          const int col0 = n0 + c * 32;
+        // stage the warp's 32 x 32 sub-tile and hand it to the TMA; rows beyond M are clipped
+        // by the tensor map
+        uint8_t* sb = my_out + (nchunk & 1) * kChunkBytes;
+        if (lane == 0) bulk_wait_group_read<1>();   // the copy that last read sb is done
+        __syncwarp();
+        const int col0 = n0 + c * 32;
+        if constexpr (kF32Out) {
+          // fp32 rows of 128 bytes, 128-byte swizzle: chunk k of row r at k ^ (r & 7)
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            v[j] = __uint_as_float(r[j]) + (bias ? __ldg(bias + col0 + j) : 0.f);
+            if (EPI == EPI_RESID && gate) v[j] *= __ldg(gate + col0 + j);
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<float4*>(sb + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        } else {
+          // bf16 rows of 64 bytes, 64-byte swizzle: chunk k of row r at k ^ ((r >> 1) & 3)
           uint32_t w[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -224,19 +194,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int k = 0; k < 4; ++k)
             *reinterpret_cast<uint4*>(sb + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)) =
                 make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (EPI == EPI_RESID)
+            tma_reduce_add_2d(&tmY, sb, col0, m0 + quarter * 32);
+          else
             tma_store_2d(&tmY, sb, col0, m0 + quarter * 32);
-            bulk_commit_group();
-          }
-        } else {
-          if (row < M) epilogue_chunk<EPI>(r, row, n0 + c * 32, Nout, bias, gate, out);
+          bulk_commit_group();
         }
       }
       if (!ok) break;
     }
-    if (kTmaOut && lane == 0) bulk_wait_group_all();
+    if (lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();
@@ -277,11 +248,12 @@ static int launch_gemm_epi(const void* A, int M, int K, const void* W, int Nout,
   if (rc) return rc;
   rc = make_tmap_2d(&tb, W, true, (uint64_t)K, (uint64_t)Nout, (uint64_t)K * 2, kGemmBK, (uint32_t)BN, true);
   if (rc) return rc;
-  CUtensorMap ty = tb;   // unused unless the output is bf16
-  if (EPI == EPI_STORE || EPI == EPI_GELU) {
+  CUtensorMap ty;   // the output, in 32 x 32 boxes: bf16 with 64-byte swizzle, fp32 with 128-byte swizzle
+  if (EPI == EPI_STORE || EPI == EPI_GELU)
     rc = make_tmap_2d_sw64(&ty, out, true, (uint64_t)Nout, (uint64_t)M, (uint64_t)Nout * 2, 32, 32);
-    if (rc) return rc;
-  }
+  else
+    rc = make_tmap_2d(&ty, out, false, (uint64_t)Nout, (uint64_t)M, (uint64_t)Nout * 4, 32, 32, true);
+  if (rc) return rc;
   if (BN == 256) return launch_gemm_bn<256, EPI>(ta, tb, ty, M, Nout, K, bias, gate, out, st);
   if (BN == 128) return launch_gemm_bn<128, EPI>(ta, tb, ty, M, Nout, K, bias, gate, out, st);
   return launch_gemm_bn<64, EPI>(ta, tb, ty, M, Nout, K, bias, gate, out, st);
