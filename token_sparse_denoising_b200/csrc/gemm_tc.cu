@@ -40,9 +40,18 @@ struct GemmCfg {
   static_assert(kSmem <= 232448, "GEMM shared memory above the 227 KB per-CTA limit");
 };
 
+// GELU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).  The tanh is the hardware
+// tanh.approx.f32 (one MUFU op, relative error about 2^-11); the result is rounded to bf16, whose
+// step is 2^-8 relative, so the approximation is below the output's own rounding.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ float gelu_tanh_f(float x) {
-  const float u = 0.7978845608028654f * (x + 0.044715f * x * x * x);
-  return 0.5f * x * (1.0f + tanhf(u));
+  const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
+  const float hx = 0.5f * x;
+  return fmaf(hx, tanh_approx(u), hx);
 }
 
 // Persistent: CTA c handles output tiles c, c + gridDim.x, ... (n fastest, so the
