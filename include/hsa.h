@@ -114,6 +114,18 @@ int hsa_select_tokens(const float* d_score, int N, int K, const int* h_group_siz
                       int8_t* d_group, int32_t* d_order, void* d_ws, size_t ws_bytes,
                       void* stream);
 
+/* The same partition with a set of pinned tokens (image-to-video, HSA summary §4: the
+ * conditioning image must stay intact, read here as its latent frame's tokens keeping the
+ * full step budget).  d_pinned[N] (uint8, device, may be NULL = none pinned): a token with
+ * d_pinned[n] != 0 ranks ahead of every unpinned token whatever its score, NaN included;
+ * pinned tokens rank among themselves by index.  So with at most n_1 pinned tokens all of
+ * them land in G_1; more than n_1 continue into G_2, ... in index order (not an error).
+ * Same outputs, workspace and errors as hsa_select_tokens, which equals this call with
+ * d_pinned = NULL.  The pages give no mechanism for I2V; this is a reading. */
+int hsa_select_tokens_pinned(const float* d_score, const uint8_t* d_pinned, int N, int K,
+                             const int* h_group_sizes, int8_t* d_group, int32_t* d_order,
+                             void* d_ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------ §2.3 cached Euler update
  * One iteration's solver update over all N tokens:
  *   1. v_hat[idx[r]] = v_A[r] for r < M (fresh velocities of A_i);

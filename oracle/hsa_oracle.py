@@ -138,7 +138,7 @@ def score_order_key(score_f32: np.ndarray) -> np.ndarray:
     return key
 
 
-def select_groups(score_f32: np.ndarray, sizes) -> tuple[np.ndarray, np.ndarray]:
+def select_groups(score_f32: np.ndarray, sizes, pinned=None) -> tuple[np.ndarray, np.ndarray]:
     """Assign tokens to groups G_1..G_K by their score (§2.1).
 
     Tokens are ranked by (score descending, index ascending); the first n_1
@@ -146,9 +146,16 @@ def select_groups(score_f32: np.ndarray, sizes) -> tuple[np.ndarray, np.ndarray]
     tokens (low L1 change) land in the groups with the fewest steps.
     Returns group[N] (int8, 0-based) and order[N]: the groups' token lists
     concatenated in group order, each list ascending by token index.
+
+    pinned (bool[N], optional): image-to-video reading of §4 (the conditioning
+    image must survive): pinned tokens rank ahead of every other token, among
+    themselves by index, so they fill G_1 first whatever their score.
     """
     key = score_order_key(score_f32)
     N = key.shape[0]
+    if pinned is not None:
+        key = key.copy()
+        key[np.asarray(pinned, bool)] = 1 << 32       # above every 32-bit order key
     ranked = np.lexsort((np.arange(N), -key))
     group = np.empty(N, dtype=np.int8)
     start = 0
@@ -379,15 +386,22 @@ def hsa_iteration(state: dict, i: int, plan: dict, velocity_fn) -> dict:
     order = state["order"]
     group = state.get("group")
     if full:
-        group, order = select_groups(score.astype(np.float32), sizes)
+        group, order = select_groups(score.astype(np.float32), sizes, plan.get("pinned"))
     return {"x": x, "v_hat": v_hat, "order": order, "group": group, "caches": caches,
             "idx": idx, "score": score, "v_A": v_A}
 
 
-def make_plan(T, budgets, sizes, m, sigma_kind, shift, N) -> dict:
+def make_plan(T, budgets, sizes, m, sigma_kind, shift, N, pinned=None) -> dict:
     validate_plan(T, budgets, sizes, N, m)
     return {"T": T, "budgets": list(budgets), "sizes": list(sizes), "m": m,
-            "sigmas": sigma_schedule(T, sigma_kind, shift), "table": active_table(T, budgets, m)}
+            "sigmas": sigma_schedule(T, sigma_kind, shift), "table": active_table(T, budgets, m),
+            "pinned": None if pinned is None else np.asarray(pinned, bool)}
+
+
+def conditioning_frame_tokens(pos: np.ndarray, n_frames: int = 1) -> np.ndarray:
+    """Image-to-video reading of §4: the tokens of the first n_frames latent frames carry the
+    conditioning image; pos is the (N, 3) (frame, row, column) table of the tokens."""
+    return np.asarray(pos)[:, 0] < n_frames
 
 
 def hsa_denoise(x0, v_hat0, plan, velocity_fn, caches0, keep_states: bool = False):

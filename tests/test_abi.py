@@ -64,6 +64,9 @@ def test_device_calls_reject_bad_arguments_on_host(lib):
     sizes = (C.c_int * 2)(4, 4)
     assert lib.hsa_select_tokens(null, 8, 0, sizes, null, null, null, 0, null) == hsa.HSA_EINVAL
     assert lib.hsa_select_tokens(null, 8, 2, (C.c_int * 2)(4, 5), null, null, null, 0, null) == hsa.HSA_EINVAL
+    assert lib.hsa_select_tokens_pinned(null, null, 8, 0, sizes, null, null, null, 0, null) == hsa.HSA_EINVAL
+    assert lib.hsa_select_tokens_pinned(null, null, 8, 2, (C.c_int * 2)(4, 5), null, null, null, 0,
+                                        null) == hsa.HSA_EINVAL
     assert lib.hsa_euler_update(null, null, null, null, 0, 8, 6, 0.1, null, null) == hsa.HSA_EINVAL
     assert lib.hsa_euler_update(null, null, null, null, 9, 8, 4, 0.1, null, null) == hsa.HSA_EINVAL
     assert lib.hsa_l1_score(null, null, 4, 3, null, null) == hsa.HSA_EINVAL

@@ -77,6 +77,29 @@ def test_select_tokens_bit_exact(cuda_lib, seed, N, K, kind):
     assert np.array_equal(host(order), want_o)
 
 
+@pytest.mark.parametrize("seed,N,K,kind,pin", [(10, 6, 3, "ties", "random"), (11, 1000, 3, "ties", "random"),
+                                               (12, 32760, 3, "rand", "first_frame"), (13, 32760, 3, "ties", "many"),
+                                               (14, 4097, 4, "const", "random"), (15, 75600, 3, "rand", "first_frame"),
+                                               (16, 1000, 2, "rand", "all"), (17, 1000, 3, "rand", "none")])
+def test_select_tokens_pinned_bit_exact(cuda_lib, seed, N, K, kind, pin):
+    """Pinned tokens (image-to-video: the conditioning frame) rank ahead of all others; compared
+    bit for bit with the oracle.  'many' pins more tokens than G_1 holds (they continue into G_2
+    by index); N = 75600 takes the unstaged path."""
+    scores, sizes = _select_case(seed, N, K, kind)
+    if K == 3 and pin in ("first_frame", "many"):
+        sizes = S.group_sizes(N, (0.25, 0.25, 0.5))
+    r = np.random.default_rng(seed + 1000)
+    pinned = {"random": r.random(N) < 0.2, "first_frame": np.arange(N) < N // 21,
+              "many": r.random(N) < 0.4, "all": np.ones(N, bool), "none": np.zeros(N, bool)}[pin]
+    group = torch.full((N,), -7, dtype=torch.int8, device="cuda")
+    order = torch.full((N,), -7, dtype=torch.int32, device="cuda")
+    cuda_lib.select_tokens(dev(scores), sizes, group, order, pinned=torch.from_numpy(pinned.astype(np.uint8)).cuda())
+    assert cuda_lib.device_status() == 0
+    want_g, want_o = O.select_groups(scores, sizes, pinned)
+    assert np.array_equal(host(group), want_g)
+    assert np.array_equal(host(order), want_o)
+
+
 # ------------------------------------------------------------------ linear layers
 
 def _lin_case(seed, M, K, Nout, bf16):

@@ -151,6 +151,70 @@ def test_selection_vs_brute_force(seed):
         start += nk
 
 
+def test_selection_pinned_hand_example():
+    rows = {r[0]: r[1:] for r in _read_rows("selection_pinned_example.txt")}
+    scores = np.array([float(v) for v in rows["scores"]], np.float32)
+    pinned = np.array([int(v) for v in rows["pinned"]], bool)
+    for case in ("a", "b"):
+        group, order = O.select_groups(scores, [int(v) for v in rows["sizes_" + case]], pinned)
+        assert list(group) == [int(v) for v in rows["group_" + case]], case
+        assert list(order) == [int(v) for v in rows["order_" + case]], case
+
+
+def _brute_rank_pinned(scores, pinned):
+    """rank(n) = #{j ranked before n}: pinned before unpinned; pinned by index; unpinned by
+    (value descending, index ascending), NaN as +inf, <= 0 as 0 (pure Python)."""
+    def val(s):
+        return math.inf if math.isnan(s) else max(float(s), 0.0)
+    vals = [val(s) for s in scores]
+
+    def before(j, n):
+        if pinned[j] != pinned[n]:
+            return bool(pinned[j])
+        if pinned[j]:
+            return j < n
+        return vals[j] > vals[n] or (vals[j] == vals[n] and j < n)
+    return [sum(1 for j in range(len(vals)) if before(j, n)) for n in range(len(vals))]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_selection_pinned_vs_brute_force(seed):
+    r = np.random.default_rng(100 + seed)
+    N = int(r.integers(1, 150))
+    scores = r.choice([0.0, 0.25, 0.5, 1.0, np.nan], size=N).astype(np.float32) if seed % 2 else \
+        r.random(N).astype(np.float32)
+    pinned = r.random(N) < (0.05, 0.3, 0.9)[seed % 3]
+    K = int(r.integers(1, 5))
+    cuts = np.sort(r.integers(0, N + 1, size=K - 1))
+    sizes = list(np.diff(np.concatenate([[0], cuts, [N]])).astype(int))
+    group, order = O.select_groups(scores, sizes, pinned)
+    rank = _brute_rank_pinned(list(scores), list(pinned))
+    bounds = np.cumsum(sizes)
+    for n in range(N):
+        assert group[n] == int(np.searchsorted(bounds, rank[n], side="right"))
+    n_pin = int(pinned.sum())
+    if n_pin <= sizes[0]:
+        assert np.all(group[pinned] == 0)          # every pinned token keeps the full budget
+
+
+def test_selection_without_pins_is_unchanged():
+    r = np.random.default_rng(7)
+    scores = r.random(90).astype(np.float32)
+    scores[::11] = np.nan
+    sizes = [30, 30, 30]
+    g0, o0 = O.select_groups(scores, sizes)
+    g1, o1 = O.select_groups(scores, sizes, np.zeros(90, bool))
+    assert np.array_equal(g0, g1) and np.array_equal(o0, o1)
+
+
+def test_conditioning_frame_tokens_are_the_first_frame():
+    grid = S.Grid(3, 2, 4)
+    pos = S.token_positions(grid)
+    mask = O.conditioning_frame_tokens(pos)
+    assert mask.sum() == 8 and np.all(np.nonzero(mask)[0] == np.arange(8))   # raster order: frame 0 first
+    assert O.conditioning_frame_tokens(pos, 2).sum() == 16
+
+
 def test_active_rows_prefix_for_nested_budgets():
     order = np.array([3, 5, 0, 2, 1, 4], np.int32)
     assert list(O.active_rows(order, [2, 2, 2], [True, True, False])) == [3, 5, 0, 2]
@@ -426,6 +490,35 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(O, "select_groups", bad_select)
     with pytest.raises(AssertionError):
         test_selection_hand_example()
+    monkeypatch.setattr(O, "select_groups", _ORIGINALS["select_groups"])
+
+    # pinned tokens given the NaN key (+inf) instead of a key above it, or ranked by score among
+    # themselves, fail the worked pinned selection
+    original_key = O.score_order_key
+
+    def pinned_as_inf(score, sizes, pinned=None):
+        s = np.array(score, np.float32)
+        if pinned is not None:
+            s[np.asarray(pinned, bool)] = np.inf
+        return _ORIGINALS["select_groups"](s, sizes)
+
+    def pinned_by_score(score, sizes, pinned=None):
+        key = original_key(score)
+        if pinned is not None:
+            key = key + np.where(np.asarray(pinned, bool), 1 << 32, 0)
+        ranked = np.lexsort((np.arange(len(key)), -key))
+        group = np.empty(len(key), np.int8)
+        start = 0
+        for k, n in enumerate(sizes):
+            group[ranked[start:start + n]] = k
+            start += n
+        order = np.concatenate([np.sort(np.nonzero(group == k)[0]) for k in range(len(sizes))])
+        return group, order
+    for bad in (pinned_as_inf, pinned_by_score):
+        monkeypatch.setattr(O, "select_groups", bad)
+        with pytest.raises(AssertionError):
+            test_selection_pinned_hand_example()
+    monkeypatch.setattr(O, "select_groups", _ORIGINALS["select_groups"])
 
 
 _ORIGINALS = {n: getattr(O, n) for n in ("rope_3d", "rms_norm", "gelu_tanh", "linear", "active_table",

@@ -3,7 +3,10 @@
 // slowest-changing tokens get the fewest denoising steps.
 //
 // Total order: (score descending, token index ascending); scores compare as
-// float32 with NaN ranking as +inf and values <= 0 as 0.  Group k holds ranks
+// float32 with NaN ranking as +inf and values <= 0 as 0.  Optionally a set of
+// pinned tokens (image-to-video: the conditioning frame's tokens) ranks ahead of
+// every other token, pinned tokens among themselves by index, so they fill G_1
+// first whatever their score.  Group k holds ranks
 // [c_{k-1}, c_k) with c_k = n_1 + ... + n_k.  The result is unique, so the GPU
 // output is compared bit for bit.
 //
@@ -74,12 +77,21 @@ __device__ int block_exclusive_scan(int v, int* total, int* warp_sums) {
 // digit at `shift` (per-warp private copies, then summed), and the digit holding the
 // element of rank `rank` among them.  Returns (digit, rank within that digit) through
 // shared memory.  Every thread of the block calls it.
-// Inverted order key of token n (ascending = descending score), from the keys staged in
-// shared memory when the kernel has them, else from the scores in global memory.
+// Inverted order key of token n (ascending = descending score): ~score_key, or 0 for a
+// pinned token (score_key never exceeds 0x7F800000, so ~0xFFFFFFFF = 0 ranks before every
+// score).  Read from the keys staged in shared memory when the kernel has them, else from
+// the scores (and pin mask) in global memory.
+__device__ __forceinline__ uint32_t inverted_key(const float* __restrict__ score, const uint8_t* __restrict__ pinned,
+                                                 int n) {
+  return (pinned && pinned[n]) ? 0u : ~score_key(score[n]);
+}
 struct KeySource {
   const float* __restrict__ score;
-  const uint32_t* ikeys;  // shared memory, or nullptr
-  __device__ __forceinline__ uint32_t operator()(int n) const { return ikeys ? ikeys[n] : ~score_key(score[n]); }
+  const uint8_t* __restrict__ pinned;  // nullable
+  const uint32_t* ikeys;               // shared memory, or nullptr
+  __device__ __forceinline__ uint32_t operator()(int n) const {
+    return ikeys ? ikeys[n] : inverted_key(score, pinned, n);
+  }
 };
 
 __device__ void radix_pass(KeySource key, int N, uint32_t mask, uint32_t prefix, int shift,
@@ -140,8 +152,8 @@ __device__ void radix_pass(KeySource key, int N, uint32_t mask, uint32_t prefix,
 }
 
 __global__ void __launch_bounds__(kSelectThreads, 1)
-    k_select(const float* __restrict__ score, int N, SelectArgs a, int8_t* __restrict__ group,
-             int* __restrict__ order) {
+    k_select(const float* __restrict__ score, const uint8_t* __restrict__ pinned, int N, SelectArgs a,
+             int8_t* __restrict__ group, int* __restrict__ order) {
   __shared__ uint32_t hw[kSelectThreads / 32][257];   // per-warp private histograms
   __shared__ uint32_t hist[256];
   __shared__ uint32_t hist0[256];                      // first-pass histogram, shared by all boundaries
@@ -154,9 +166,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
   const int tid = threadIdx.x;
   const int chunk = (N + kSelectThreads - 1) / kSelectThreads;
   const int lo = min(N, tid * chunk), hi = min(N, lo + chunk);
-  KeySource key{score, nullptr};
+  KeySource key{score, pinned, nullptr};
   if (a.staged) {
-    for (int n = tid; n < N; n += kSelectThreads) s_ikeys[n] = ~score_key(score[n]);
+    for (int n = tid; n < N; n += kSelectThreads) s_ikeys[n] = inverted_key(score, pinned, n);
     __syncthreads();
     key.ikeys = s_ikeys;
   }
@@ -285,8 +297,9 @@ extern "C" size_t hsa_select_tokens_workspace_size(int N, int K) {
   return 0;
 }
 
-extern "C" int hsa_select_tokens(const float* d_score, int N, int K, const int* h_group_sizes, int8_t* d_group,
-                                 int32_t* d_order, void* d_ws, size_t ws_bytes, void* stream) {
+extern "C" int hsa_select_tokens_pinned(const float* d_score, const uint8_t* d_pinned, int N, int K,
+                                        const int* h_group_sizes, int8_t* d_group, int32_t* d_order, void* d_ws,
+                                        size_t ws_bytes, void* stream) {
   using namespace hsa;
   (void)d_ws;
   (void)ws_bytes;
@@ -316,7 +329,12 @@ extern "C" int hsa_select_tokens(const float* d_score, int N, int K, const int* 
     attr_done[dev] = true;
   }
   ScopedTiming timing(HSA_KCLASS_OTHER, as_stream(stream));
-  k_select<<<1, kSelectThreads, dyn, as_stream(stream)>>>(d_score, N, a, d_group, d_order);
+  k_select<<<1, kSelectThreads, dyn, as_stream(stream)>>>(d_score, d_pinned, N, a, d_group, d_order);
   count_launch(1);
   return check_launch("select launch");
+}
+
+extern "C" int hsa_select_tokens(const float* d_score, int N, int K, const int* h_group_sizes, int8_t* d_group,
+                                 int32_t* d_order, void* d_ws, size_t ws_bytes, void* stream) {
+  return hsa_select_tokens_pinned(d_score, nullptr, N, K, h_group_sizes, d_group, d_order, d_ws, ws_bytes, stream);
 }

@@ -47,6 +47,7 @@ _SIGS = {
     "hsa_l1_score": (i32, [vp, vp, i32, i32, vp, vp]),
     "hsa_select_tokens_workspace_size": (sz, [i32, i32]),
     "hsa_select_tokens": (i32, [vp, i32, i32, vp, vp, vp, vp, sz, vp]),
+    "hsa_select_tokens_pinned": (i32, [vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
     "hsa_euler_update": (i32, [vp, vp, vp, vp, i32, i32, i32, f32, vp, vp]),
     "hsa_context_kv_workspace_size": (sz, [i32, i32]),
     "hsa_context_kv": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -170,7 +171,9 @@ def select_tokens_workspace_size(N: int, K: int) -> int:
     return int(lib().hsa_select_tokens_workspace_size(N, K))
 
 
-def select_tokens(score, group_sizes, group, order, stream=None, ws=None):
+def select_tokens(score, group_sizes, group, order, stream=None, ws=None, pinned=None):
+    """Group partition by score; `pinned` (uint8 [N] on the device, optional) ranks those tokens
+    ahead of all others (hsa_select_tokens_pinned)."""
     import torch
     N = score.shape[0]
     K = len(group_sizes)
@@ -180,8 +183,15 @@ def select_tokens(score, group_sizes, group, order, stream=None, ws=None):
         ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=score.device)
     elif ws.numel() * ws.element_size() < nbytes:
         raise ValueError("select_tokens: workspace smaller than hsa_select_tokens_workspace_size")
-    _check(lib().hsa_select_tokens(_ptr(score), N, K, sizes.ctypes.data, _ptr(group), _ptr(order), _ptr(ws),
-                                   nbytes, _stream(stream)), "hsa_select_tokens")
+    if pinned is None:
+        _check(lib().hsa_select_tokens(_ptr(score), N, K, sizes.ctypes.data, _ptr(group), _ptr(order), _ptr(ws),
+                                       nbytes, _stream(stream)), "hsa_select_tokens")
+    else:
+        if pinned.dtype != torch.uint8 or pinned.numel() != N:
+            raise ValueError("select_tokens: pinned must be a uint8 tensor of N entries")
+        _check(lib().hsa_select_tokens_pinned(_ptr(score), _ptr(pinned), N, K, sizes.ctypes.data, _ptr(group),
+                                              _ptr(order), _ptr(ws), nbytes, _stream(stream)),
+               "hsa_select_tokens_pinned")
 
 
 def euler_update(x, vhat, vA, idx, dsigma: float, score=None, stream=None):

@@ -102,11 +102,20 @@ class PatchModel:
         return vA
 
 
+def conditioning_frame_mask(pos, n_frames: int = 1) -> np.ndarray:
+    """Image-to-video: the tokens of the first n_frames latent frames (the conditioning image),
+    from the (N, 3) (frame, row, column) position table.  Pass it as HSARun(pinned=...)."""
+    return np.asarray(pos)[:, 0] < n_frames
+
+
 class HSARun:
-    """Latent x, cached velocities v_hat and the token grouping of one run, plus its schedule."""
+    """Latent x, cached velocities v_hat and the token grouping of one run, plus its schedule.
+
+    pinned (bool[N], optional): tokens kept in G_1 at every regrouping whatever their score
+    (image-to-video: conditioning_frame_mask); see hsa_select_tokens_pinned."""
 
     def __init__(self, model, x0, vhat0, T: int, budgets, sizes, m: int, sigma_kind: int, shift: float,
-                 device="cuda"):
+                 device="cuda", pinned=None):
         self.model = model
         N = x0.shape[0]
         self.N, self.T, self.sizes = N, T, list(sizes)
@@ -118,6 +127,8 @@ class HSARun:
         self.group = torch.zeros(N, dtype=torch.int8, device=device)
         self.score = torch.zeros(N, dtype=torch.float32, device=device)
         self.idx_buf = torch.empty(N, dtype=torch.int32, device=device)
+        self.pinned = None if pinned is None else \
+            torch.from_numpy(np.ascontiguousarray(pinned, bool).astype(np.uint8)).to(device)
         self.sel_ws = torch.empty(max(hsa.select_tokens_workspace_size(N, len(self.sizes)), 1), dtype=torch.uint8,
                                   device=device)
         self.starts = np.concatenate([[0], np.cumsum(self.sizes)]).astype(np.int64)
@@ -174,7 +185,7 @@ class HSARun:
         dsig = float(np.float32(self.sigmas[i + 1]) - np.float32(self.sigmas[i]))
         hsa.euler_update(self.x, self.vhat, vA, idx, dsig, score=self.score if full else None)
         if full:
-            hsa.select_tokens(self.score, self.sizes, self.group, self.order, ws=self.sel_ws)
+            hsa.select_tokens(self.score, self.sizes, self.group, self.order, ws=self.sel_ws, pinned=self.pinned)
         if record is not None:
             record.append({"i": i, "M": int(idx.shape[0]), "full": full,
                            "score": self.score.cpu().numpy().copy() if full else None,
