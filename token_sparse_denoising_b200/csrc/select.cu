@@ -17,8 +17,12 @@
 //      top-digit pass is shared by all boundaries), then the right index among
 //      the equal keys by a block scan;
 //   2. each token's group = number of boundaries it ranks at or after;
-//   3. the groups' lists, each ascending by index, by per-thread chunk counts
-//      and one block scan per group; group k starts at c_{k-1}.
+//   3. the groups' lists, each ascending by index: warp w owns a contiguous index
+//      range and walks it 32 consecutive indices at a time (bank-conflict-free
+//      shared-memory reads, coalesced writes); per-group warp counts come from
+//      ballots, one scan over the warps per group gives each warp its offsets,
+//      and a lane's position is the number of lower lanes in its group.  Group k
+//      starts at c_{k-1}.
 // For N <= 40960 the order keys are first staged in shared memory, so the passes
 // do not wait on L2 latency for every element.
 #include "common.cuh"
@@ -158,14 +162,18 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
   __shared__ uint32_t hist[256];
   __shared__ uint32_t hist0[256];                      // first-pass histogram, shared by all boundaries
   __shared__ int warp_sums[33];
+  __shared__ int s_wcnt[kMaxGroups][kSelectThreads / 32];   // per group, per warp: count, then offset
   __shared__ uint32_t s_thr_key[kMaxGroups];
   __shared__ int s_thr_idx[kMaxGroups];
   __shared__ int s_digit, s_rank;
   extern __shared__ uint32_t s_ikeys[];                // N staged keys when the launch provides them
 
-  const int tid = threadIdx.x;
-  const int chunk = (N + kSelectThreads - 1) / kSelectThreads;
-  const int lo = min(N, tid * chunk), hi = min(N, lo + chunk);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = kSelectThreads / 32;
+  // warp w owns indices [wlo, whi): a multiple of 32 per warp, walked 32 consecutive at a time
+  const int per_warp = ((N + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int wlo = min(N, warp * per_warp), whi = min(N, wlo + per_warp);
+  const unsigned lanes_below = (1u << lane) - 1u;
   KeySource key{score, pinned, nullptr};
   if (a.staged) {
     for (int n = tid; n < N; n += kSelectThreads) s_ikeys[n] = inverted_key(score, pinned, n);
@@ -224,68 +232,109 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
       rank = s_rank;
       __syncthreads();
     }
-    // the rank-th smallest token index among keys equal to the target
+    // the rank-th smallest token index among keys equal to the target: per-warp counts of
+    // matches, a scan over the warps, then the warp holding that rank finds the lane
     int cnt = 0;
-    for (int n = lo; n < hi; ++n) cnt += (key(n) == prefix);
-    int total;
-    const int excl = block_exclusive_scan(cnt, &total, warp_sums);
-    if (rank >= excl && rank < excl + cnt) {
+    for (int base = wlo; base < whi; base += 32) {
+      const int n = base + lane;
+      cnt += __popc(__ballot_sync(0xffffffffu, n < whi && key(n) == prefix));
+    }
+    if (lane == 0) warp_sums[warp] = cnt;
+    __syncthreads();
+    if (warp == 0) {
+      const int v = warp_sums[lane];
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      warp_sums[lane] = incl - v;
+    }
+    __syncthreads();
+    const int excl = warp_sums[warp];
+    if (rank >= excl && rank < excl + cnt) {      // warp-uniform
       int seen = excl;
-      for (int n = lo; n < hi; ++n) {
-        if (key(n) == prefix) {
-          if (seen == rank) {
+      for (int base = wlo; base < whi; base += 32) {
+        const int n = base + lane;
+        const bool m = n < whi && key(n) == prefix;
+        const unsigned mk = __ballot_sync(0xffffffffu, m);
+        if (rank < seen + __popc(mk)) {
+          if (m && seen + __popc(mk & lanes_below) == rank) {
             s_thr_idx[b] = n;
             s_thr_key[b] = ~prefix;
-            break;
           }
-          ++seen;
+          break;
         }
+        seen += __popc(mk);
       }
     }
     __syncthreads();
   }
 
-  // ---- 2. group of each token in this thread's chunk; local counts per group.  Loops over
-  // groups are unrolled to kMaxGroups with a K guard, so cnt[] and off[] stay in registers.
+  // ---- 2. group of each token; per-warp counts per group.  Loops over groups are unrolled to
+  // kMaxGroups with a K guard, so the counters stay in registers (warp-uniform values).
   int cnt[kMaxGroups];
 #pragma unroll
   for (int k = 0; k < kMaxGroups; ++k) cnt[k] = 0;
-  for (int n = lo; n < hi; ++n) {
-    const uint32_t kn = ~key(n);
-    int g = 0;
+  for (int base = wlo; base < whi; base += 32) {
+    const int n = base + lane;
+    const bool valid = n < whi;
+    int g = -1;
+    if (valid) {
+      const uint32_t kn = ~key(n);
+      g = 0;
 #pragma unroll
-    for (int b = 1; b < kMaxGroups; ++b) {
-      if (b < a.K) {
-        const int c = a.cum[b];
-        if (c <= 0) {
-          ++g;
-        } else if (c < N) {
-          const uint32_t kt = s_thr_key[b];
-          if (kn < kt || (kn == kt && n > s_thr_idx[b])) ++g;
+      for (int b = 1; b < kMaxGroups; ++b) {
+        if (b < a.K) {
+          const int c = a.cum[b];
+          if (c <= 0) {
+            ++g;
+          } else if (c < N) {
+            const uint32_t kt = s_thr_key[b];
+            if (kn < kt || (kn == kt && n > s_thr_idx[b])) ++g;
+          }
         }
       }
+      group[n] = (int8_t)g;
+      if (key.ikeys) s_ikeys[n] = (uint32_t)g;   // this lane's own slot: it now holds the group
     }
-    group[n] = (int8_t)g;
-    if (key.ikeys) s_ikeys[n] = (uint32_t)g;   // this thread's own slot: it now holds the group
-#pragma unroll
-    for (int k = 0; k < kMaxGroups; ++k) cnt[k] += (g == k);
-  }
-
-  // ---- 3. ascending per-group lists, group k starting at cum[k]
-  int off[kMaxGroups];
-#pragma unroll
-  for (int k = 0; k < kMaxGroups; ++k) {
-    off[k] = 0;
-    if (k < a.K) {  // uniform over the block: every thread takes the same scans
-      int total;
-      off[k] = a.cum[k] + block_exclusive_scan(cnt[k], &total, warp_sums);
-    }
-  }
-  for (int n = lo; n < hi; ++n) {
-    const int g = key.ikeys ? (int)s_ikeys[n] : (int)group[n];
 #pragma unroll
     for (int k = 0; k < kMaxGroups; ++k)
-      if (k == g) order[off[k]++] = n;
+      if (k < a.K) cnt[k] += __popc(__ballot_sync(0xffffffffu, g == k));
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int k = 0; k < kMaxGroups; ++k)
+      if (k < a.K) s_wcnt[k][warp] = cnt[k];
+  }
+  __syncthreads();
+  // ---- 3. offsets: warp k scans group k's counts over the warps (ascending index ranges)
+  if (warp < a.K) {
+    const int v = s_wcnt[warp][lane];
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    s_wcnt[warp][lane] = a.cum[warp] + incl - v;
+  }
+  __syncthreads();
+  int off[kMaxGroups];
+#pragma unroll
+  for (int k = 0; k < kMaxGroups; ++k) off[k] = (k < a.K) ? s_wcnt[k][warp] : 0;
+  for (int base = wlo; base < whi; base += 32) {
+    const int n = base + lane;
+    const int g = n < whi ? (key.ikeys ? (int)s_ikeys[n] : (int)group[n]) : -1;
+#pragma unroll
+    for (int k = 0; k < kMaxGroups; ++k) {
+      if (k < a.K) {
+        const unsigned mk = __ballot_sync(0xffffffffu, g == k);
+        if (g == k) order[off[k] + __popc(mk & lanes_below)] = n;
+        off[k] += __popc(mk);
+      }
+    }
   }
 }
 
