@@ -405,11 +405,14 @@ def run_sweep(args):
             q = torch.randn((M, 1536), device="cuda").to(torch.bfloat16)
             o = torch.empty_like(q)
             reps = 5
+            need = hsa.attention_workspace_size(M, N, 12, hsa.HSA_BF16)
+            ws = torch.empty(need, dtype=torch.uint8, device="cuda") if need else None
             for _ in range(2):
-                hsa.attention(q, k, v, 12, o)
-            ms = time_device(lambda: hsa.attention(q, k, v, 12, o), reps, lambda: None) / reps
+                hsa.attention(q, k, v, 12, o, ws=ws)
+            ms = time_device(lambda: hsa.attention(q, k, v, 12, o, ws=ws), reps, lambda: None) / reps
             tf = 4.0 * M * N * 128 * 12 / (ms * 1e-3) / 1e12
-            res["attention"].append({"N": N, "frac": f, "M": M, "ms": round(ms, 4), "tflops": round(tf, 1),
+            res["attention"].append({"N": N, "frac": f, "M": M, "split_ws_bytes": int(need), "ms": round(ms, 4),
+                                     "tflops": round(tf, 1),
                                      "frac_of_burst_peak": round(tf / peak_burst, 3)})
         x = torch.randn((N, 64), device="cuda")
         vh = torch.randn((N, 64), device="cuda")

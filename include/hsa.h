@@ -206,7 +206,10 @@ int hsa_context_kv_noalloc(const void* d_ctx, int L, int D, int dtype, const voi
  * d_x_src: when not NULL, X is first gathered as d_x_src[idx[r]] (N x D float32)
  *   and written to d_xA; when NULL, d_xA already holds X.
  * d_idx: M distinct token indices in [0, N); d_pos: N x 3 int32 (frame, row, column).
- * 1 <= M <= N.  Workspace: hsa_layer_step_workspace_size(M, D, F, dtype). */
+ * 1 <= M <= N.  Workspace: hsa_layer_step_workspace_size(M, D, F, dtype).  A workspace sized
+ * for a larger M (say N, reused for every step) leaves room the attention uses to split the
+ * key range of its last, incomplete wave of work units (see hsa_attention_ws); results agree
+ * with the unsplit path to rounding. */
 size_t hsa_layer_step_workspace_size(int M, int D, int F, int dtype);
 int hsa_layer_step(const hsa_layer_weights* w, void* d_kcache, void* d_vcache, int N, float* d_xA,
                    const float* d_x_src, const int32_t* d_idx, int M, const int32_t* d_pos,
@@ -219,6 +222,20 @@ int hsa_layer_step(const hsa_layer_weights* w, void* d_kcache, void* d_vcache, i
  *   d_q: M x 128H, d_k, d_v: L x 128H, d_o: M x 128H, all in dtype. */
 int hsa_attention(const void* d_q, int M, const void* d_k, const void* d_v, int L, int H, int dtype,
                   void* d_o, void* stream);
+
+/* The same attention with a workspace.  The work units are (128-query tile, head) pairs, one
+ * per SM at a time.  The units that fill complete waves of the GPU's SMs run whole.  With
+ * ws_bytes >= hsa_attention_workspace_size(M, L, H, dtype), each unit of the last, incomplete
+ * wave is split over S ranges of key tiles, so the split CTAs fill that wave.  Each split
+ * writes an unnormalised fp32 output and its row max and sum to d_ws, and a second kernel
+ * merges them:
+ *   o = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s,  m = max_s m_s.
+ * A smaller or NULL workspace runs every unit whole, like hsa_attention.  Only the bf16 path
+ * splits; the size is 0 when no split pays off (every wave complete, or fewer than 4 key tiles).
+ * d_ws must be 16-byte aligned.  Not in the pages: a scheduling choice of this implementation. */
+size_t hsa_attention_workspace_size(int M, int L, int H, int dtype);
+int hsa_attention_ws(const void* d_q, int M, const void* d_k, const void* d_v, int L, int H, int dtype,
+                     void* d_o, void* d_ws, size_t ws_bytes, void* stream);
 
 /* Linear layer on compacted rows: y = epilogue(x W^T + b) for x: M x Kin (dtype),
  * W: [Nout][Kin] (dtype), b: [Nout] float32 (NULL = 0).

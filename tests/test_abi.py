@@ -102,3 +102,14 @@ def test_binding_fails_loudly_without_library(tmp_path):
             hsa.load(str(tmp_path / "libhsa.so"))
     finally:
         hsa._lib = saved
+
+
+def test_attention_workspace_size_follows_the_last_wave(lib):
+    """The split scratch is sized only when the last wave of (query tile, head) units is
+    incomplete and worth splitting (148 SMs assumed without a device)."""
+    bf, f32 = hsa.HSA_BF16, hsa.HSA_F32
+    assert lib.hsa_attention_workspace_size(32760, 32760, 12, bf) == 0      # 3072 units: no split pays
+    assert lib.hsa_attention_workspace_size(8190, 32760, 12, bf) > 0        # 768 units: 28 in the tail
+    assert lib.hsa_attention_workspace_size(8190, 32760, 12, f32) == 0
+    assert lib.hsa_attention_workspace_size(300, 256, 2, bf) == 0           # 2 key tiles: nothing to split
+    assert lib.hsa_attention_workspace_size(0, 100, 2, bf) == 0

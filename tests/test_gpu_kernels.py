@@ -183,6 +183,52 @@ def test_attention_identical_keys_give_mean_value(cuda_lib):
     assert max_abs(host(o), np.tile(v.astype(np.float64).mean(0), (M, 1))) < 1e-2
 
 
+@pytest.mark.parametrize("M,L,H", [(1000, 4000, 12), (300, 1000, 2), (300, 512, 2), (129, 2000, 3)])
+def test_attention_split_tail_matches_oracle(cuda_lib, M, L, H):
+    """With a workspace the units of the last, incomplete wave are split over key ranges and
+    merged by a second kernel (1000 x 4000 x 12 heads: 96 units, 3 ranges each; 300 x 1000: the
+    last range holds the ragged key tile; 300 x 512: ranges of two tiles).  Checked against the
+    oracle, and against the unsplit kernel to fp32-merge rounding."""
+    D = 128 * H
+    q = S.normal(71, (M, D), 1.0, True)
+    k, v = S.normal(72, (L, D), 1.0, True), S.normal(73, (L, D), 1.0, True)
+    need = cuda_lib.attention_workspace_size(M, L, H, cuda_lib.HSA_BF16)
+    assert need > 0                                    # these shapes do split
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    o = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    o1 = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    qd, kd, vd = dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16)
+    cuda_lib.attention(qd, kd, vd, H, o, ws=ws)
+    cuda_lib.attention(qd, kd, vd, H, o1)
+    assert cuda_lib.device_status() == 0
+    assert_bf16_close(host(o), O.attention(q, k, v), "split attention")
+    assert max_abs(host(o), host(o1)) <= 2 ** -7          # at most a bf16 step apart
+    # a workspace one byte short runs every unit whole: bit-identical to hsa_attention
+    short = torch.empty(need - 1, dtype=torch.uint8, device="cuda")
+    o2 = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    cuda_lib.attention(qd, kd, vd, H, o2, ws=short)
+    assert torch.equal(o2, o1)
+
+
+def test_attention_split_tail_wan_quarter(cuda_lib):
+    """The Wan-1.3B shape at |A|/N = 1/4 (8190 queries, 32760 keys, 12 heads): 768 units, the 28
+    of the incomplete last wave split 5 ways; sampled rows against the oracle."""
+    M, L, H = 8190, 32760, 12
+    D = 128 * H
+    q = S.normal(81, (M, D), 1.0, True)
+    k, v = S.normal(82, (L, D), 1.0, True), S.normal(83, (L, D), 1.0, True)
+    need = cuda_lib.attention_workspace_size(M, L, H, cuda_lib.HSA_BF16)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    o = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    cuda_lib.attention(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), H, o, ws=ws)
+    assert cuda_lib.device_status() == 0
+    # rows of whole units, of split units (tail = units 740..767: heads 11 and 12 of the tiles), ragged end
+    rows = np.array([0, 1, 4000, 7000, 7424, 7900, 8100, 8189])
+    got = host(o)[rows]
+    want = O.attention(q[rows], k, v)
+    assert_bf16_close(got, want, "split attention, sampled rows")
+
+
 @pytest.mark.parametrize("M,L,H", [(100, 300, 2), (1, 1024, 1)])
 def test_attention_f32(cuda_lib, M, L, H):
     D = 128 * H

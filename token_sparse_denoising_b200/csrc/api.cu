@@ -10,11 +10,12 @@ int gemm_bf16(const void* A, int M, int K, const void* W, int Nout, const float*
               void* out, cudaStream_t st);
 int gemm_f32(const float* A, int M, int K, const float* W, int Nout, const float* bias, int epi, const float* gate,
              float* out, cudaStream_t st);
-int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, int H, void* O, cudaStream_t st);
+int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, int H, void* O, cudaStream_t st,
+                   void* ws, size_t ws_bytes);
+size_t attention_split_bytes(int M, int L, int H);
 int attention_f32(const float* Q, int M, const float* K, const float* V, int L, int H, float* O, cudaStream_t st);
 
 static inline unsigned warp_blocks(long long rows) { return (unsigned)((rows * 32 + 255) / 256); }
-static inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 static inline size_t esize(int dtype) { return dtype == HSA_BF16 ? 2 : 4; }
 
 #define HSA_TRY(x)            \
@@ -76,9 +77,10 @@ static int linear(const void* x, int M, int K, const void* W, int Nout, const fl
                   static_cast<float*>(y), st);
 }
 
+// ws (may be null): scratch for splitting the tail units of the bf16 kernel over key ranges
 static int attention(const void* q, int M, const void* k, const void* v, int L, int H, int dtype, void* o,
-                     cudaStream_t st) {
-  if (dtype == HSA_BF16) return attention_bf16(q, M, k, v, L, H, o, st);
+                     cudaStream_t st, void* ws = nullptr, size_t ws_bytes = 0) {
+  if (dtype == HSA_BF16) return attention_bf16(q, M, k, v, L, H, o, st, ws, ws_bytes);
   return attention_f32(static_cast<const float*>(q), M, static_cast<const float*>(k),
                        static_cast<const float*>(v), L, H, static_cast<float*>(o), st);
 }
@@ -142,6 +144,18 @@ extern "C" int hsa_attention(const void* d_q, int M, const void* d_k, const void
   if (dtype != HSA_BF16 && dtype != HSA_F32) return set_error(HSA_EINVAL, "attention: unknown dtype");
   if (M < 0) return set_error(HSA_EINVAL, "attention: M < 0");
   return attention(d_q, M, d_k, d_v, L, H, dtype, d_o, as_stream(stream));
+}
+
+extern "C" size_t hsa_attention_workspace_size(int M, int L, int H, int dtype) {
+  return dtype == HSA_BF16 ? attention_split_bytes(M, L, H) : 0;
+}
+
+extern "C" int hsa_attention_ws(const void* d_q, int M, const void* d_k, const void* d_v, int L, int H, int dtype,
+                                void* d_o, void* d_ws, size_t ws_bytes, void* stream) {
+  if (dtype != HSA_BF16 && dtype != HSA_F32) return set_error(HSA_EINVAL, "attention: unknown dtype");
+  if (M < 0) return set_error(HSA_EINVAL, "attention: M < 0");
+  if (d_ws && !aligned16(d_ws)) return set_error(HSA_EINVAL, "attention: misaligned workspace");
+  return attention(d_q, M, d_k, d_v, L, H, dtype, d_o, as_stream(stream), d_ws, ws_bytes);
 }
 
 // ------------------------------------------------------------------ §2.2 context keys / values
@@ -224,6 +238,10 @@ extern "C" int hsa_layer_step(const hsa_layer_weights* w, void* d_kcache, void* 
 
   cudaStream_t st = as_stream(stream);
   StepWs ws = carve_step_ws(d_ws, M, D, F, dt);
+  // the FFN hidden region and whatever the caller's workspace has beyond it are free until the
+  // FFN: the attention calls may use them to split their tail over key ranges
+  void* spare = ws.hid;
+  const size_t spare_bytes = ws_bytes - (size_t)(static_cast<uint8_t*>(ws.hid) - static_cast<uint8_t*>(d_ws));
   const float* mod = w->mod;
   const bool bf = dt == HSA_BF16;
   using bf16 = __nv_bfloat16;
@@ -241,7 +259,7 @@ extern "C" int hsa_layer_step(const hsa_layer_weights* w, void* d_kcache, void* 
                            static_cast<float*>(ws.q), static_cast<float*>(d_kcache), static_cast<float*>(d_vcache),
                            st));
   // a3: full-context attention over all N cache rows
-  HSA_TRY(attention(ws.q, M, d_kcache, d_vcache, N, H, dt, ws.att, st));
+  HSA_TRY(attention(ws.q, M, d_kcache, d_vcache, N, H, dt, ws.att, st, spare, spare_bytes));
   // a4: gated output projection into the residual stream
   HSA_TRY(linear(ws.att, M, D, w->w_o, D, w->b_o, dt, HSA_EPI_RESID, mod + 2 * D, d_xA, st));
   if (cross) {
@@ -250,7 +268,7 @@ extern "C" int hsa_layer_step(const hsa_layer_weights* w, void* d_kcache, void* 
     HSA_TRY(linear(ws.h, M, D, w->w_q2, D, w->b_q2, dt, HSA_EPI_STORE, nullptr, ws.qkv, st));
     if (bf) HSA_TRY(launch_rms(static_cast<const bf16*>(ws.qkv), D, M, D, w->g_q2, static_cast<bf16*>(ws.q), st));
     else HSA_TRY(launch_rms(static_cast<const float*>(ws.qkv), D, M, D, w->g_q2, static_cast<float*>(ws.q), st));
-    HSA_TRY(attention(ws.q, M, d_ctx_k, d_ctx_v, ctx_len, H, dt, ws.att, st));
+    HSA_TRY(attention(ws.q, M, d_ctx_k, d_ctx_v, ctx_len, H, dt, ws.att, st, spare, spare_bytes));
     HSA_TRY(linear(ws.att, M, D, w->w_o2, D, w->b_o2, dt, HSA_EPI_RESID, nullptr, d_xA, st));
   }
   // a4: gated GELU feed-forward

@@ -31,6 +31,12 @@
 // execute in issue order.
 // Key rows beyond L are zero-filled by TMA and masked to -inf; query rows beyond
 // M are computed on zeros and never stored.
+//
+// Work units are (128-query tile, head) pairs, one per CTA, in blockIdx.x order.  The
+// units of the complete waves run whole.  When a workspace is given, the units of an
+// incomplete last wave are each split over S ranges of key tiles (S chosen so the split
+// CTAs fill the last wave).  A split CTA writes its unnormalised O (fp32) with its row
+// max and sum, and k_attn_combine merges the S parts into the bf16 output.
 #include "tcgen05.cuh"
 
 namespace hsa {
@@ -60,6 +66,16 @@ struct AttnShared {
   float xm[2][128], xl[2][128];  // [parity][row]: running max and sum, merged in the epilogue
 };
 constexpr int kAttnSmem = kTileBytes * (1 + kKSlots + kVSlots) + 1024 + (int)sizeof(AttnShared);
+
+// Unit -> CTA map: units u < u_full are whole; unit u_full + t / s_tail, key range t % s_tail,
+// for the split tail.  part_o / part_ml hold the split CTAs' partial results, slot t.
+struct AttnGrid {
+  int QT;          // query tiles per head
+  int u_full;      // units run whole
+  int s_tail;      // key-range splits of each tail unit (1: no split)
+  float* part_o;   // [slots][128][128] unnormalised O
+  float2* part_ml; // [slots][128] (row max in log2 units, row sum)
+};
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -113,7 +129,8 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, int M, int L, int H, __nv_bfloat16* __restrict__ O) {
+              const __grid_constant__ CUtensorMap tmV, int M, int L, int H, __nv_bfloat16* __restrict__ O,
+              const AttnGrid grid) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -122,8 +139,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   AttnShared* sh = reinterpret_cast<AttnShared*>(sV + kVSlots * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kAttnBM, h = blockIdx.y;
-  const int nj = (L + kAttnBN - 1) / kAttnBN;
+  int u = blockIdx.x, split = 0, n_split = 1, slot = -1;
+  if (u >= grid.u_full) {
+    const int t = u - grid.u_full;
+    u = grid.u_full + t / grid.s_tail;
+    split = t % grid.s_tail;
+    n_split = grid.s_tail;
+    if (n_split > 1) slot = t;
+  }
+  const int m0 = (u % grid.QT) * kAttnBM, h = u / grid.QT;
+  // this CTA's key tiles [j0, j0 + nj): loops, ring slots and parities use the local index
+  const int nj_all = (L + kAttnBN - 1) / kAttnBN;
+  const int j0 = split * nj_all / n_split;
+  const int nj = (split + 1) * nj_all / n_split - j0;
 
   if (threadIdx.x == 0) {
     mbar_init(&sh->q_full, 1);
@@ -170,8 +198,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ok && leader) {
         uint8_t* k = sK + sk * kTileBytes;
         mbar_expect_tx(&sh->k_full[sk], kTileBytes);
-        tma_load_2d(k, &tmK, &sh->k_full[sk], x0, j * kAttnBN);
-        tma_load_2d(k + kTileBytes / 2, &tmK, &sh->k_full[sk], x0 + 64, j * kAttnBN);
+        tma_load_2d(k, &tmK, &sh->k_full[sk], x0, (j0 + j) * kAttnBN);
+        tma_load_2d(k + kTileBytes / 2, &tmK, &sh->k_full[sk], x0 + 64, (j0 + j) * kAttnBN);
       }
       return ok;
     };
@@ -185,8 +213,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (leader) {
         uint8_t* v = sV + sv * kTileBytes;
         mbar_expect_tx(&sh->v_full[sv], kTileBytes);
-        tma_load_2d(v, &tmV, &sh->v_full[sv], x0, j * kAttnBN);
-        tma_load_2d(v + kTileBytes / 2, &tmV, &sh->v_full[sv], x0 + 64, j * kAttnBN);
+        tma_load_2d(v, &tmV, &sh->v_full[sv], x0, (j0 + j) * kAttnBN);
+        tma_load_2d(v + kTileBytes / 2, &tmV, &sh->v_full[sv], x0 + 64, (j0 + j) * kAttnBN);
       }
       if (j + 2 < nj) ok = load_k(j + 2);
     }
@@ -265,8 +293,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld32(s_col + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + q4 * 32));
       tmem_ld_wait();
 
-      if ((j + 1) * kAttnBN > L) {  // ragged last tile only: keys beyond L get -inf
-        const int valid = L - j * kAttnBN;
+      if ((j0 + j + 1) * kAttnBN > L) {  // ragged last tile only: keys beyond L get -inf
+        const int valid = L - (j0 + j) * kAttnBN;
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
@@ -344,6 +372,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
     tc_fence_after();
     const int grow = m0 + row;
+    if (slot >= 0) {
+      // split CTA: unnormalised O relative to mm, and (mm, a0 l_0 + a1 l_1), for k_attn_combine
+      float* dst_o = grid.part_o + ((size_t)slot * kAttnBM + row) * 128;
+      if (par == 0) grid.part_ml[(size_t)slot * kAttnBM + row] = make_float2(mm, a0 * sh->xl[0][row] + a1 * sh->xl[1][row]);
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        const uint32_t col = (uint32_t)(par * 64 + c * 32);
+        uint32_t o0[32], o1[32];
+        __syncwarp();
+        tmem_ld32(lane_base + kColO + col, o0);
+        if (two) tmem_ld32(lane_base + kColO + 128 + col, o1);
+        tmem_ld_wait();
+        if (!two) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o1[e] = 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst_o + col + e) =
+              make_float4(fmaf(__uint_as_float(o0[e + 0]), a0, __uint_as_float(o1[e + 0]) * a1),
+                          fmaf(__uint_as_float(o0[e + 1]), a0, __uint_as_float(o1[e + 1]) * a1),
+                          fmaf(__uint_as_float(o0[e + 2]), a0, __uint_as_float(o1[e + 2]) * a1),
+                          fmaf(__uint_as_float(o0[e + 3]), a0, __uint_as_float(o1[e + 3]) * a1));
+      }
+    } else {
     // this warp writes output columns [par * 64, par * 64 + 64) of the head
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
@@ -364,14 +417,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           float f[8];
 #pragma unroll
           for (int t = 0; t < 8; ++t) f[t] = fmaf(__uint_as_float(o0[e + t]), w0, __uint_as_float(o1[e + t]) * w1);
-          uint4 u;
-          u.x = pack_bf16x2(f[0], f[1]);
-          u.y = pack_bf16x2(f[2], f[3]);
-          u.z = pack_bf16x2(f[4], f[5]);
-          u.w = pack_bf16x2(f[6], f[7]);
-          *reinterpret_cast<uint4*>(dst + e) = u;
+          uint4 pk4;
+          pk4.x = pack_bf16x2(f[0], f[1]);
+          pk4.y = pack_bf16x2(f[2], f[3]);
+          pk4.z = pack_bf16x2(f[4], f[5]);
+          pk4.w = pack_bf16x2(f[6], f[7]);
+          *reinterpret_cast<uint4*>(dst + e) = pk4;
         }
       }
+    }
     }
   }
 
@@ -384,7 +438,78 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, int H, void* O, cudaStream_t st) {
+// Merge the key-range splits of the tail units: one warp per (tail unit, row), lane = 4 channels.
+//   O = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s,  m = max_s m_s.
+__global__ void __launch_bounds__(256) k_attn_combine(const float* __restrict__ part_o,
+                                                      const float2* __restrict__ part_ml, int n_tail, int s_tail,
+                                                      int u_full, int QT, int M, int H,
+                                                      __nv_bfloat16* __restrict__ O) {
+  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int tu = w / kAttnBM, row = w % kAttnBM;
+  if (tu >= n_tail) return;
+  const int u = u_full + tu;
+  const int grow = (u % QT) * kAttnBM + row, h = u / QT;
+  if (grow >= M) return;
+  float mx = -INFINITY;
+  for (int sp = 0; sp < s_tail; ++sp) mx = fmaxf(mx, part_ml[(size_t)(tu * s_tail + sp) * kAttnBM + row].x);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f;
+  for (int sp = 0; sp < s_tail; ++sp) {
+    const size_t r = (size_t)(tu * s_tail + sp) * kAttnBM + row;
+    const float2 ml = part_ml[r];
+    const float a = exp2f(ml.x - mx);
+    den = fmaf(a, ml.y, den);
+    const float4 o = *reinterpret_cast<const float4*>(part_o + r * 128 + lane * 4);
+    acc = make_float4(fmaf(a, o.x, acc.x), fmaf(a, o.y, acc.y), fmaf(a, o.z, acc.z), fmaf(a, o.w, acc.w));
+  }
+  const float inv = 1.0f / den;
+  uint2 pk;
+  pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  *reinterpret_cast<uint2*>(O + (size_t)grow * (H * 128) + h * 128 + lane * 4) = pk;
+}
+
+namespace {
+struct TailSplit {
+  int u_full, s_tail, n_tail;   // s_tail == 1: no split
+};
+// Units of the complete waves run whole; the n_tail units of an incomplete last wave are split
+// over S key ranges, S minimising the tail's time ceil(n_tail S / SMs) / S (in whole-unit times)
+// plus a small per-split cost (each split CTA refills the pipeline).  Each split keeps at least
+// two key tiles, and a split is taken only when it saves at least 15 % of the tail's time.
+TailSplit plan_tail(int U, int nj_all, int sms) {
+  TailSplit p{U, 1, 0};
+  const int tail = U % sms;
+  if (tail == 0) return p;
+  int best_s = 1;
+  double best = 0.85;
+  for (int S = 2; S <= 16 && 2 * S <= nj_all; ++S) {
+    const double t = (double)((tail * S + sms - 1) / sms) / S + 0.02 * S;
+    if (t < best - 1e-9) {
+      best = t;
+      best_s = S;
+    }
+  }
+  if (best_s == 1) return p;
+  return TailSplit{U - tail, best_s, tail};
+}
+size_t tail_split_bytes(const TailSplit& p) {
+  if (p.s_tail <= 1) return 0;
+  const size_t slots = (size_t)p.n_tail * p.s_tail * kAttnBM;
+  return align256(slots * 128 * sizeof(float)) + align256(slots * sizeof(float2));
+}
+}  // namespace
+
+size_t attention_split_bytes(int M, int L, int H) {
+  if (M <= 0 || L <= 0 || H <= 0) return 0;
+  const int QT = (M + kAttnBM - 1) / kAttnBM;
+  return tail_split_bytes(plan_tail(QT * H, (L + kAttnBN - 1) / kAttnBN, num_sms()));
+}
+
+// bf16 attention; with a workspace of at least attention_split_bytes(M, L, H) the tail units
+// are split over key ranges (otherwise, or with none, every unit runs whole).
+int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, int H, void* O, cudaStream_t st,
+                   void* ws, size_t ws_bytes) {
   if (M <= 0) return HSA_OK;
   if (L <= 0 || H <= 0) return set_error(HSA_EINVAL, "attention: need L > 0 and H > 0");
   if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
@@ -404,10 +529,29 @@ int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, in
       return check_launch("attention: shared-memory attribute");
     attr_done[dev] = true;
   }
+  const int QT = (M + kAttnBM - 1) / kAttnBM, U = QT * H;
+  TailSplit ts = plan_tail(U, (L + kAttnBN - 1) / kAttnBN, num_sms());
+  const size_t need = tail_split_bytes(ts);
+  if (need == 0 || !ws || ws_bytes < need || !aligned16(ws)) ts = TailSplit{U, 1, 0};
+  AttnGrid g{QT, ts.u_full, ts.s_tail, nullptr, nullptr};
+  if (ts.s_tail > 1) {
+    const size_t slots = (size_t)ts.n_tail * ts.s_tail * kAttnBM;
+    g.part_o = static_cast<float*>(ws);
+    g.part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + align256(slots * 128 * sizeof(float)));
+  }
   ScopedTiming timing(HSA_KCLASS_ATTENTION, st);
-  dim3 grid((M + kAttnBM - 1) / kAttnBM, H);
-  k_attn_tc<<<grid, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, M, L, H, reinterpret_cast<__nv_bfloat16*>(O));
+  const int ctas = ts.u_full + ts.n_tail * ts.s_tail;
+  k_attn_tc<<<ctas, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, M, L, H, reinterpret_cast<__nv_bfloat16*>(O), g);
   count_launch(1);
+  if (ts.s_tail > 1) {
+    rc = check_launch("attn_tc launch");
+    if (rc) return rc;
+    const int warps = ts.n_tail * kAttnBM;
+    k_attn_combine<<<(warps + 7) / 8, 256, 0, st>>>(g.part_o, g.part_ml, ts.n_tail, ts.s_tail, ts.u_full, QT, M, H,
+                                                     reinterpret_cast<__nv_bfloat16*>(O));
+    count_launch(1);
+    return check_launch("attn_combine launch");
+  }
   return check_launch("attn_tc launch");
 }
 

@@ -39,5 +39,6 @@ class ScopedTiming {
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 }  // namespace hsa

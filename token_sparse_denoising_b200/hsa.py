@@ -56,6 +56,8 @@ _SIGS = {
     "hsa_layer_step_workspace_size": (sz, [i32, i32, i32, i32]),
     "hsa_layer_step": (i32, [C.POINTER(LayerWeightsC), vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, i32, vp, sz, vp]),
     "hsa_attention": (i32, [vp, i32, vp, vp, i32, i32, i32, vp, vp]),
+    "hsa_attention_workspace_size": (sz, [i32, i32, i32, i32]),
+    "hsa_attention_ws": (i32, [vp, i32, vp, vp, i32, i32, i32, vp, vp, sz, vp]),
     "hsa_linear": (i32, [vp, i32, i32, vp, i32, vp, i32, i32, vp, vp, vp]),
     "hsa_patch_workspace_size": (sz, [i32, i32, i32, i32]),
     "hsa_patch_embed": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]),
@@ -207,9 +209,20 @@ def linear(x, w, b, epilogue: int, y, gate=None, stream=None):
                             _ptr(y), _stream(stream)), "hsa_linear")
 
 
-def attention(q, k, v, H: int, o, stream=None):
-    _check(lib().hsa_attention(_ptr(q), q.shape[0], _ptr(k), _ptr(v), k.shape[0], H, _dtype_code(q), _ptr(o),
-                               _stream(stream)), "hsa_attention")
+def attention(q, k, v, H: int, o, stream=None, ws=None):
+    """o = softmax(q k^T / sqrt(128)) v per head; with `ws` (uint8 device tensor of at least
+    attention_workspace_size bytes) the last wave's units are split over key ranges."""
+    if ws is None:
+        _check(lib().hsa_attention(_ptr(q), q.shape[0], _ptr(k), _ptr(v), k.shape[0], H, _dtype_code(q), _ptr(o),
+                                   _stream(stream)), "hsa_attention")
+    else:
+        _check(lib().hsa_attention_ws(_ptr(q), q.shape[0], _ptr(k), _ptr(v), k.shape[0], H, _dtype_code(q),
+                                      _ptr(o), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+               "hsa_attention_ws")
+
+
+def attention_workspace_size(M: int, L: int, H: int, dtype: int) -> int:
+    return int(lib().hsa_attention_workspace_size(M, L, H, dtype))
 
 
 def context_kv_workspace_size(L: int, D: int) -> int:
