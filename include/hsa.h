@@ -63,6 +63,14 @@ const char* hsa_last_error_string(void);
  * current device: HSA_OK, HSA_EINDEX or HSA_ETIMEOUT (the first fault seen). */
 int hsa_device_status(void* stream);
 
+/* Diagnostic, not part of the method: launches one warp that waits on an mbarrier no thread
+ * ever completes.  The library's bounded wait gives up after its limit (1 s), records
+ * HSA_ETIMEOUT in the device status word and raises the abort flag that makes every pending
+ * wait of the library return at once; hsa_device_status() then returns HSA_ETIMEOUT and clears
+ * both, after which the library runs normally.  Lets a test exercise the failure path of the
+ * pipelined kernels without faulting or hanging the GPU.  Returns the launch status. */
+int hsa_selftest_wait_timeout(void* stream);
+
 /* Number of kernel launches the library has enqueued in this process. */
 uint64_t hsa_launch_count(void);
 

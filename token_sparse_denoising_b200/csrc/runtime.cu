@@ -179,6 +179,25 @@ extern "C" const char* hsa_last_error_string(void) { return hsa::t_last_error.c_
 
 extern "C" uint64_t hsa_launch_count(void) { return hsa::g_launches.load(); }
 
+// One warp waits on a shared-memory mbarrier that no thread ever arrives at: every lane's
+// bounded wait gives up after kWaitLimitNs, the first one records HSA_ETIMEOUT and raises the
+// abort flag, and the kernel returns.  Checks the failure path without a GPU fault.
+__global__ void k_wait_never() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    hsa::mbar_init(&bar, 1);
+    hsa::fence_mbar_init();
+  }
+  __syncthreads();
+  (void)hsa::mbar_wait(&bar, 0);
+}
+
+extern "C" int hsa_selftest_wait_timeout(void* stream) {
+  k_wait_never<<<1, 32, 0, hsa::as_stream(stream)>>>();
+  hsa::count_launch(1);
+  return hsa::check_launch("selftest wait launch");
+}
+
 extern "C" int hsa_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(hsa::as_stream(stream));
   if (e != cudaSuccess) return hsa::set_error(HSA_ECUDA, std::string("stream sync: ") + cudaGetErrorString(e));

@@ -39,6 +39,7 @@ class LayerWeightsC(C.Structure):
 _SIGS = {
     "hsa_last_error_string": (C.c_char_p, []),
     "hsa_device_status": (i32, [vp]),
+    "hsa_selftest_wait_timeout": (i32, [vp]),
     "hsa_launch_count": (u64, []),
     "hsa_timing_enable": (i32, [i32]),
     "hsa_timing_read": (i32, [i32, C.POINTER(C.c_double), C.POINTER(i32)]),
@@ -140,6 +141,11 @@ def plan_groups(T: int, budgets, group_sizes, N: int, m: int, sigma_kind: int, s
 
 def device_status(stream=None) -> int:
     return lib().hsa_device_status(_stream(stream))
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    """Diagnostic: a kernel whose bounded wait runs out (see hsa_selftest_wait_timeout)."""
+    _check(lib().hsa_selftest_wait_timeout(_stream(stream)), "hsa_selftest_wait_timeout")
 
 
 def launch_count() -> int:
