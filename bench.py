@@ -47,7 +47,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_traffic.json")
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=30)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["hsa", "reference"], default="hsa")
     p.add_argument("--no-sweep", action="store_true")
@@ -85,40 +85,60 @@ def synthetic_inputs():
 # ---------------------------------------------------------------- clocks during the timed region
 
 class ClockSampler:
+    """nvidia-smi polled every 50 ms from before the warm-up; stop() keeps the samples whose
+    timestamps fall inside the timed region (host clock window set by mark_start / mark_end)."""
+
     def __init__(self, index: int):
         self.path = tempfile.mktemp(suffix=".csv")
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+        self.t0 = self.t1 = None
+        q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.5)                    # let nvidia-smi start sampling before the work
         except OSError:
             self.proc = None
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def stop(self):
+        import datetime
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         self.proc.wait(timeout=10)
-        sm, mx, reasons = [], None, set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             f = [v.strip() for v in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[2]), float(f[3]), float(f[4]),
+                             [n for n, v in zip(names, f[6:10]) if v.lower() == "active"]))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
         os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        window = "timed region"
+        sel = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= self.t1]
+        if len(sel) < 2:                        # a very short timed region: add the warm-up just before it
+            window = "warm-up and timed region"
+            sel = [r for r in rows if self.t0 is not None and self.t0 - 1.0 <= r[0] <= self.t1]
+        if not sel:
+            window, sel = "whole run", rows
+        reasons = sorted({n for r in sel for n in r[4]})
+        return {"sm_mhz": statistics.median(r[1] for r in sel) if sel else None,
+                "sm_max_mhz": sel[-1][2] if sel else None, "reasons": reasons,
+                "power_w_median": statistics.median(r[3] for r in sel) if sel else None,
+                "samples": len(sel), "window": window}
 
 
 # ---------------------------------------------------------------- the CUDA path
@@ -269,17 +289,21 @@ def run_gpu(args, rank, world, barrier, allmax):
     device = torch.device("cuda", torch.cuda.current_device())
     inp = synthetic_inputs()
     step = Step(inp, device)
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     for _ in range(args.warmup):
         step.full()
     torch.cuda.synchronize()
     assert hsa.device_status() == 0, "device status after warm-up"
 
     # ---- timed region: K full iterations, per-kernel-class events on
-    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     hsa.timing_reset()
     hsa.timing_enable(True)
     l0 = hsa.launch_count()
+    if clocks:
+        clocks.mark_start()
     ms = time_device(step.full, args.steps, barrier)
+    if clocks:
+        clocks.mark_end()
     launches = hsa.launch_count() - l0
     hsa.timing_enable(False)
     attn_ms, attn_n = hsa.timing_read(hsa.KCLASS_ATTENTION)
