@@ -53,9 +53,10 @@ def parse():
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--mode", choices=["step", "loop", "sweep", "wan14"], default="step",
+    p.add_argument("--mode", choices=["step", "loop", "sweep", "wan14", "tiny"], default="step",
                    help="step: the headline line; loop: 30-block Wan-1.3B loop, HSA vs uniform 40 steps; "
-                        "sweep: attention + Euler kernel sweep; wan14: Wan-14B block active-fraction sweep")
+                        "sweep: attention + Euler kernel sweep; wan14: Wan-14B block active-fraction sweep; "
+                        "tiny: the fp32 parity workload as a whole run")
     return p.parse_args()
 
 
@@ -412,6 +413,55 @@ def run_loop(args):
     return out
 
 
+def run_tiny(args):
+    """The tiny fp32 parity workload as a whole run: 4x16x16 tokens, D = 256, one block, T = 8, budgets
+    {8, 4} at 50/50 %, m = 1 (fp32 on the CUDA cores: a parity configuration, reported in ms only).
+    Timed eagerly and as one recorded CUDA graph, against the uniform 8-step run."""
+    import torch
+    from token_sparse_denoising_b200 import hsa, pipeline
+    hsa.load()
+    wl = S.TINY_FP32
+    N, D = wl.grid.N, wl.shape.D
+    bw = S.block_weights(wl.seed, wl.shape, False)
+    pos = S.token_positions(wl.grid)
+    x0, vh0 = S.normal(wl.seed * 10 + 1, (N, D)), S.normal(wl.seed * 10 + 2, (N, D))
+    model = pipeline.SingleBlockModel(bw, pos, N, bf16=False)
+    out = {"mode": "tiny", "workload": f"{wl.name}: N={N} (4x16x16) D={D} H=2 F=1024 fp32, T={wl.T}, m={wl.m}"}
+    for name, budgets, fracs in (("hsa", wl.budgets, wl.fracs), ("uniform", (wl.T,), (1.0,))):
+        sizes = S.group_sizes(N, fracs)
+        run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift)
+        run.run()                                      # warm-up run
+        times = []
+        for _ in range(5):
+            run.reset(x0, vh0)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            run.run()
+            b.record()
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        run.reset(x0, vh0)
+        g = run.capture()
+        gtimes = []
+        for _ in range(5):
+            run.reset(x0, vh0)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            run.replay(g)
+            b.record()
+            b.synchronize()
+            gtimes.append(a.elapsed_time(b))
+        del g
+        assert hsa.device_status() == 0
+        out[name] = {"ms": round(statistics.median(times), 3), "graph_ms": round(statistics.median(gtimes), 3),
+                     "token_steps": int(run.n_active.sum())}
+    out["speedup"] = round(out["uniform"]["ms"] / out["hsa"]["ms"], 3)
+    out["speedup_graph"] = round(out["uniform"]["graph_ms"] / out["hsa"]["graph_ms"], 3)
+    return out
+
+
 def run_sweep(args):
     """Attention at N in {8190, 32760, 75600} x |A|/N in {1, .5, .25, .125} (12 heads, random active rows)
     and the Euler update on N x 64 fp32 latents."""
@@ -609,7 +659,7 @@ def main():
     torch.cuda.set_device(local)
     if args.mode != "step":
         if rank == 0:
-            fn = {"loop": run_loop, "sweep": run_sweep, "wan14": run_wan14}[args.mode]
+            fn = {"loop": run_loop, "sweep": run_sweep, "wan14": run_wan14, "tiny": run_tiny}[args.mode]
             print(json.dumps(fn(args)), flush=True)
         return 0
     dist = None
