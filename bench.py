@@ -345,12 +345,15 @@ def run_gpu(args, rank, world, barrier, allmax):
         "roofline": {"bound": "tensor", "kernel": "k_attn_tc (self + cross attention launches)",
                      "achieved": round(achieved, 1), "peak": peak_sus, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_sus, 4),
-                     "peak_note": f"{src} sustained bf16 (burst {peak_burst}: frac {achieved / peak_burst:.3f})",
+                     "peak_note": f"{src} sustained bf16 (burst {peak_burst}: frac {achieved / peak_burst:.3f}; "
+                                  f"datasheet dense bf16 2250: frac {achieved / 2250.0:.3f})",
                      "traffic": traffic, "launches_per_step": attn_n // max(args.steps, 1),
                      "flops_per_step": attn_flops_per_full_step()},
         "breakdown_ms_per_step": {"attention": round(attn_per_step, 4), "gemm": round(gemm_ms / args.steps, 4),
                                   "other": round(other_ms / args.steps, 4)},
         "sweep_ms": {k: round(v, 4) for k, v in sweep.items()},
+        "whole_job": {"replicas": world, "layer_steps_per_s": round(world * 1000.0 / ms_step, 2),
+                      "note": "independent replicas, one per rank; value is the max over ranks of ms per step"},
         "gpu_launches": int(launches),
         "clocks": clk,
         "e2e": e2e,
