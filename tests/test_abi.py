@@ -113,3 +113,56 @@ def test_attention_workspace_size_follows_the_last_wave(lib):
     assert lib.hsa_attention_workspace_size(8190, 32760, 12, f32) == 0
     assert lib.hsa_attention_workspace_size(300, 256, 2, bf) == 0           # 2 key tiles: nothing to split
     assert lib.hsa_attention_workspace_size(0, 100, 2, bf) == 0
+
+
+def _c_decls():
+    """(name, return type, [parameter types]) of every function declared in include/hsa.h."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = []
+    for m in re.finditer(r"([A-Za-z_][A-Za-z0-9_ \*]*?)\b(hsa_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        ret, name, params = m.group(1).strip(), m.group(2), " ".join(m.group(3).split())
+        plist = [] if params in ("", "void") else [p.strip() for p in params.split(",")]
+        out.append((name, ret, plist))
+    return out
+
+
+def _kind(c_type: str) -> str:
+    t = c_type.strip()
+    if "*" in t:
+        return "ptr"
+    base = t.replace("const", "").split()[0]
+    return {"int": "i32", "size_t": "u64", "float": "f32", "uint64_t": "u64"}[base]   # LP64: size_t is 64-bit
+
+
+def _ctype_kind(ct) -> str:
+    if ct in (C.c_void_p, C.c_char_p) or getattr(ct, "__name__", "").startswith("LP_"):
+        return "ptr"
+    return {C.c_int: "i32", C.c_size_t: "u64", C.c_float: "f32", C.c_uint64: "u64"}[ct]
+
+
+def test_binding_signatures_match_the_header():
+    """Every declared entry point has a binding signature with the same parameter kinds and
+    return kind, so the Python side cannot drift from the C ABI."""
+    decls = _c_decls()
+    assert len(decls) >= 20
+    for name, ret, params in decls:
+        assert name in hsa._SIGS, f"{name} missing from the binding"
+        rtype, argtypes = hsa._SIGS[name]
+        want = [_kind(p.rsplit(" ", 1)[0] if not p.endswith("*") else p) for p in params]
+        got = [_ctype_kind(a) for a in argtypes]
+        assert got == want, f"{name}: binding {got} vs header {want}"
+        want_ret = "ptr" if "*" in ret else _kind(ret)
+        assert _ctype_kind(rtype) == want_ret, f"{name}: return {rtype} vs {ret}"
+
+
+def test_layer_weights_struct_matches_the_header():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    body = re.search(r"typedef struct hsa_layer_weights \{(.*?)\} hsa_layer_weights;", text, flags=re.S).group(1)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        names = decl.split(None, 1)[1] if not decl.startswith("const") else decl.split(None, 2)[2]
+        fields += [n.strip().lstrip("*").strip() for n in names.split(",")]
+    assert fields == [f[0] for f in hsa.LayerWeightsC._fields_]
