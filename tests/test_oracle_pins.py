@@ -350,6 +350,39 @@ def test_all_active_block_equals_dense_torch_block(cross):
     assert np.allclose(K2, kref, atol=1e-10) and np.allclose(V2, vref, atol=1e-10)
 
 
+def _torch_patch_model(pm, x, pos, ctx):
+    """The all-active patch model composed from torch float64 library ops: patch embedding,
+    the blocks (each the dense torch block), LayerNorm + (shift, scale) head, D -> C."""
+    X = F.linear(_t(x), _t(pm.w_in), _t(pm.b_in)).numpy()
+    for bw in pm.blocks:
+        X = _torch_block(bw, X, pos, ctx)[0]
+    hm = _t(pm.head_mod)
+    h = F.layer_norm(_t(X), (X.shape[1],), eps=1e-6) * (1.0 + hm[1]) + hm[0]
+    return F.linear(h, _t(pm.w_out), _t(pm.b_out)).numpy()
+
+
+def test_patch_model_all_active_equals_torch_composition():
+    """The loop workload's velocity model: with every token active the oracle's patch model equals
+    the torch composition (patch embedding, dense blocks, modulated LayerNorm head)."""
+    shape = S.BlockShape(256, 2, 512, True, 16)
+    pm = S.patch_model_weights(3, shape, 64, 2, bf16=False, std=0.2)
+    pm.blocks = [S.perturb_vectors(bw, 30 + i) for i, bw in enumerate(pm.blocks)]
+    pm.b_in = S.normal(41, pm.b_in.shape, 0.3)
+    pm.b_out = S.normal(42, pm.b_out.shape, 0.3)
+    pm.head_mod = S.normal(43, pm.head_mod.shape, 0.3)
+    grid = S.Grid(2, 4, 5)
+    pos = S.token_positions(grid)
+    N = grid.N
+    x = S.normal(44, (N, 64))
+    ctx = S.normal(45, (16, 256))
+    idx = np.arange(N)
+    caches = [(S.normal(46 + b, (N, 256)), S.normal(50 + b, (N, 256))) for b in range(2)]
+    ctx_kvs = [O.context_kv(bw, ctx) for bw in pm.blocks]
+    v, _ = O.patch_model_active(pm, x, idx, pos, caches, ctx_kvs)
+    ref = _torch_patch_model(pm, x, pos, ctx)
+    assert np.allclose(v, ref, atol=1e-10)
+
+
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_gather_form_equals_mask_form(seed):
     """Brute force on N = 64 tokens (1x8x8): gather form == mask form to fp64 round-off."""
@@ -519,6 +552,14 @@ def test_planted_mistakes_are_caught(monkeypatch):
         with pytest.raises(AssertionError):
             test_selection_pinned_hand_example()
     monkeypatch.setattr(O, "select_groups", _ORIGINALS["select_groups"])
+
+    # a velocity head without its (shift, scale) modulation fails the patch-model composition
+    original_head = O.head_projection
+    monkeypatch.setattr(O, "head_projection",
+                        lambda pm, X: O.linear(O.layer_norm(X), pm.w_out, pm.b_out))
+    with pytest.raises(AssertionError):
+        test_patch_model_all_active_equals_torch_composition()
+    monkeypatch.setattr(O, "head_projection", original_head)
 
 
 _ORIGINALS = {n: getattr(O, n) for n in ("rope_3d", "rms_norm", "gelu_tanh", "linear", "active_table",
