@@ -28,14 +28,18 @@ QKV with RMSNorm on q/k, 3D RoPE (44/42/42 channel split per 128-wide head),
 softmax attention, gated output projection, optional cross-attention against
 a text context, gated GELU(tanh) feed-forward.
 
-Readings of what the pages leave open (each one is listed in the design doc):
+Readings of what the pages leave open:
   * iteration index i is 0-based, i in [0, T); step i moves sigma_i -> sigma_{i+1};
   * groups are ranked by (score descending, token index ascending); group 1
     takes the highest scores; scores are compared as float32, NaN as +inf;
   * L1 relative change = sum_c |v_new - v_prev| / (sum_c |v_prev| + 1e-8);
   * selection re-runs after every step in which all N tokens were active;
   * the cache holds post-RMSNorm, post-RoPE K, and V;
-  * compacted active rows are the groups' ascending index lists in group order.
+  * compacted active rows are the groups' ascending index lists in group order;
+  * image-to-video (§4 reports only the outcome): the conditioning frame's
+    tokens are pinned ahead of every score, so they keep the full budget;
+  * a static grouping (a fixed partition, never regrouped) is the plainest
+    alternative to the dynamic selection.
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py
 except the model-level quality of HSA itself (parity unpinned: the pages give
@@ -385,17 +389,31 @@ def hsa_iteration(state: dict, i: int, plan: dict, velocity_fn) -> dict:
     x, v_hat = cached_euler(state["x"], state["v_hat"], v_A, idx, dsig)
     order = state["order"]
     group = state.get("group")
-    if full:
+    if full and plan.get("static_groups") is None:
         group, order = select_groups(score.astype(np.float32), sizes, plan.get("pinned"))
     return {"x": x, "v_hat": v_hat, "order": order, "group": group, "caches": caches,
             "idx": idx, "score": score, "v_A": v_A}
 
 
-def make_plan(T, budgets, sizes, m, sigma_kind, shift, N, pinned=None) -> dict:
+def make_plan(T, budgets, sizes, m, sigma_kind, shift, N, pinned=None, static_groups=None) -> dict:
+    """static_groups (int[N], optional): a fixed partition for the whole run (token n in group
+    static_groups[n]; group k must hold sizes[k] tokens) instead of regrouping by score after full
+    steps -- the plainest static alternative to the dynamic selection of §2.1."""
     validate_plan(T, budgets, sizes, N, m)
+    if static_groups is not None:
+        g = np.asarray(static_groups, np.int64)
+        if g.shape != (N,) or [int(np.sum(g == k)) for k in range(len(sizes))] != list(sizes):
+            raise ValueError("static groups must give group k exactly sizes[k] tokens")
     return {"T": T, "budgets": list(budgets), "sizes": list(sizes), "m": m,
             "sigmas": sigma_schedule(T, sigma_kind, shift), "table": active_table(T, budgets, m),
-            "pinned": None if pinned is None else np.asarray(pinned, bool)}
+            "pinned": None if pinned is None else np.asarray(pinned, bool),
+            "static_groups": None if static_groups is None else np.asarray(static_groups, np.int64)}
+
+
+def static_order(static_groups, K: int) -> np.ndarray:
+    """The groups' token lists of a fixed partition, concatenated in group order, each ascending."""
+    g = np.asarray(static_groups, np.int64)
+    return np.concatenate([np.nonzero(g == k)[0] for k in range(K)]).astype(np.int32)
 
 
 def conditioning_frame_tokens(pos: np.ndarray, n_frames: int = 1) -> np.ndarray:
@@ -408,11 +426,13 @@ def hsa_denoise(x0, v_hat0, plan, velocity_fn, caches0, keep_states: bool = Fals
     """The whole loop: T iterations of hsa_iteration from x0 with cached velocities v_hat0.
 
     The order before step 0 is the identity (step 0 is always a full step, so
-    it never decides which tokens run).
+    it never decides which tokens run); with static groups it is their fixed order.
     """
     N = x0.shape[0]
+    order0 = np.arange(N, dtype=np.int32) if plan.get("static_groups") is None else \
+        static_order(plan["static_groups"], len(plan["sizes"]))
     state = {"x": np.asarray(x0, F64), "v_hat": np.asarray(v_hat0, F64),
-             "order": np.arange(N, dtype=np.int32), "group": None, "caches": caches0}
+             "order": order0, "group": None, "caches": caches0}
     states = []
     for i in range(plan["T"]):
         state = hsa_iteration(state, i, plan, velocity_fn)

@@ -112,6 +112,42 @@ def test_tiny_fp32_loop_matches_oracle(cuda_lib):
     assert_f32_close(x_gpu[keep] - x0[keep], final["x"][keep] - x0[keep], "latent displacement")
 
 
+@pytest.mark.parametrize("pattern", ["frames", "checkerboard"])
+def test_tiny_fp32_loop_static_groups_match_oracle_on_every_token(cuda_lib, pattern):
+    """The tiny fp32 loop with a static partition (never regrouped): no selection, so no near-ties,
+    and the whole run is compared with the oracle on every token.  'frames': frames 0-1 in G_1,
+    2-3 in G_2; 'checkerboard': alternate (row + column) parity, so the group lists interleave."""
+    wl = S.TINY_FP32
+    N, D = wl.grid.N, wl.shape.D
+    bw = S.block_weights(wl.seed, wl.shape, False)
+    pos = S.token_positions(wl.grid)
+    x0, vh0 = S.normal(wl.seed * 10 + 1, (N, D)), S.normal(wl.seed * 10 + 2, (N, D))
+    sizes = S.group_sizes(N, wl.fracs)
+    if pattern == "frames":
+        groups = (pos[:, 0] >= 2).astype(np.int64)
+    else:
+        groups = ((pos[:, 1] + pos[:, 2]) % 2).astype(np.int64)
+    model = pipeline.SingleBlockModel(bw, pos, N, bf16=False)
+    run = pipeline.HSARun(model, x0, vh0, wl.T, wl.budgets, sizes, wl.m, wl.sigma_kind, wl.shift,
+                          static_groups=groups)
+    rec = []
+    x_gpu = host(run.run(rec))
+    assert hsa.device_status() == 0
+
+    plan = O.make_plan(wl.T, wl.budgets, sizes, wl.m, wl.sigma_kind, wl.shift, N, static_groups=groups)
+
+    def vel(xA, idx, caches):
+        out, Kc, Vc = O.dit_block_active(bw, xA, idx, pos, caches[0], caches[1])
+        return out, (Kc, Vc)
+
+    zeros = np.zeros((N, D))
+    final, states = O.hsa_denoise(x0, vh0, plan, vel, (zeros, zeros), keep_states=True)
+    for r, st in zip(rec, states):
+        assert r["M"] == len(st["idx"]) and np.array_equal(r["order"], st["order"])
+    assert_f32_close(x_gpu, final["x"], "final latent")
+    assert_f32_close(x_gpu - x0, final["x"] - x0, "latent displacement")
+
+
 def test_tiny_fp32_loop_image_to_video_pins(cuda_lib):
     """The tiny fp32 loop with the first frame's 256 tokens pinned to G_1 (image-to-video reading).
     After step 0 this random block's scores fall into two clusters of near-equal values (a token's

@@ -215,6 +215,24 @@ def test_conditioning_frame_tokens_are_the_first_frame():
     assert O.conditioning_frame_tokens(pos, 2).sum() == 16
 
 
+def test_static_groups_never_regroup():
+    """With a fixed partition every full step keeps the order; the active rows of each step are the
+    fixed groups' lists; a partition with the wrong sizes is rejected."""
+    N, T = 12, 4
+    groups = np.array([1, 0, 1, 0, 0, 1, 1, 0, 1, 0, 0, 1])
+    plan = O.make_plan(T, [4, 2], [6, 6], 1, 0, 1.0, N, static_groups=groups)
+    order = O.static_order(groups, 2)
+    assert list(order) == [1, 3, 4, 7, 9, 10, 0, 2, 5, 6, 8, 11]
+    model = lambda xA, idx, c: (xA * 0.5 + idx[:, None], c)
+    x0, vh0 = np.ones((N, 4)), np.zeros((N, 4))
+    _, states = O.hsa_denoise(x0, vh0, plan, model, None, keep_states=True)
+    for i, st in enumerate(states):
+        assert list(st["order"]) == list(order)
+        assert list(st["idx"]) == (list(order) if i in (0, 2, 3) else list(order[:6]))
+    with pytest.raises(ValueError):
+        O.make_plan(T, [4, 2], [6, 6], 1, 0, 1.0, N, static_groups=np.zeros(N, int))
+
+
 def test_active_rows_prefix_for_nested_budgets():
     order = np.array([3, 5, 0, 2, 1, 4], np.int32)
     assert list(O.active_rows(order, [2, 2, 2], [True, True, False])) == [3, 5, 0, 2]

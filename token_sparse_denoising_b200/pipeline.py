@@ -112,10 +112,12 @@ class HSARun:
     """Latent x, cached velocities v_hat and the token grouping of one run, plus its schedule.
 
     pinned (bool[N], optional): tokens kept in G_1 at every regrouping whatever their score
-    (image-to-video: conditioning_frame_mask); see hsa_select_tokens_pinned."""
+    (image-to-video: conditioning_frame_mask); see hsa_select_tokens_pinned.
+    static_groups (int[N], optional): a fixed partition for the whole run (token n in group
+    static_groups[n], group k holding sizes[k] tokens); full steps then do not regroup."""
 
     def __init__(self, model, x0, vhat0, T: int, budgets, sizes, m: int, sigma_kind: int, shift: float,
-                 device="cuda", pinned=None):
+                 device="cuda", pinned=None, static_groups=None):
         self.model = model
         N = x0.shape[0]
         self.N, self.T, self.sizes = N, T, list(sizes)
@@ -123,7 +125,14 @@ class HSARun:
                                                                  shift)
         self.x = _to_dev(x0, torch.float32, device)
         self.vhat = _to_dev(vhat0, torch.float32, device)
-        self.order = torch.arange(N, dtype=torch.int32, device=device)
+        self.static_order = None
+        if static_groups is not None:
+            g = np.asarray(static_groups, np.int64)
+            if g.shape != (N,) or [int(np.sum(g == k)) for k in range(len(self.sizes))] != self.sizes:
+                raise ValueError("static groups must give group k exactly sizes[k] tokens")
+            self.static_order = np.concatenate([np.nonzero(g == k)[0] for k in range(len(self.sizes))])
+        self.order = torch.arange(N, dtype=torch.int32, device=device) if self.static_order is None else \
+            torch.from_numpy(self.static_order.astype(np.int32)).to(device)
         self.group = torch.zeros(N, dtype=torch.int8, device=device)
         self.score = torch.zeros(N, dtype=torch.float32, device=device)
         self.idx_buf = torch.empty(N, dtype=torch.int32, device=device)
@@ -139,7 +148,8 @@ class HSARun:
         the loop can be replayed for a new latent."""
         self.x.copy_(torch.as_tensor(np.ascontiguousarray(x0, np.float32)))
         self.vhat.copy_(torch.as_tensor(np.ascontiguousarray(vhat0, np.float32)))
-        self.order.copy_(torch.arange(self.N, dtype=torch.int32))
+        self.order.copy_(torch.arange(self.N, dtype=torch.int32) if self.static_order is None else
+                         torch.from_numpy(self.static_order.astype(np.int32)))
         self.group.zero_()
         self.score.zero_()
         self.i = 0
@@ -183,12 +193,13 @@ class HSARun:
         full = idx.shape[0] == self.N
         vA = self.model.velocity(self.x, idx)
         dsig = float(np.float32(self.sigmas[i + 1]) - np.float32(self.sigmas[i]))
-        hsa.euler_update(self.x, self.vhat, vA, idx, dsig, score=self.score if full else None)
-        if full:
+        regroup = full and self.static_order is None
+        hsa.euler_update(self.x, self.vhat, vA, idx, dsig, score=self.score if regroup else None)
+        if regroup:
             hsa.select_tokens(self.score, self.sizes, self.group, self.order, ws=self.sel_ws, pinned=self.pinned)
         if record is not None:
             record.append({"i": i, "M": int(idx.shape[0]), "full": full,
-                           "score": self.score.cpu().numpy().copy() if full else None,
+                           "score": self.score.cpu().numpy().copy() if regroup else None,
                            "order": self.order.cpu().numpy().copy()})
         self.i += 1
 
