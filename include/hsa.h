@@ -134,6 +134,15 @@ int hsa_select_tokens_pinned(const float* d_score, const uint8_t* d_pinned, int 
                              const int* h_group_sizes, int8_t* d_group, int32_t* d_order,
                              void* d_ws, size_t ws_bytes, void* stream);
 
+/* A_i for iteration i (§2.1): the lists of the groups active at i, taken from d_order (the
+ * groups' lists concatenated in group order, as hsa_select_tokens writes it), concatenated in
+ * group order into d_idx[M], M = sum of the active groups' sizes (written to *h_M when h_M is
+ * not NULL).  h_active[K]: 1 for a group running at i (a row of hsa_plan_groups' table).  With
+ * nested budgets A_i is a prefix of d_order and needs no copy; this call covers every other
+ * pattern with one launch.  HSA_EINVAL when the sizes do not sum to N or K is out of range. */
+int hsa_active_rows(const int32_t* d_order, int N, int K, const int* h_group_sizes,
+                    const uint8_t* h_active, int32_t* d_idx, int* h_M, void* stream);
+
 /* ------------------------------------------------------------------ §2.3 cached Euler update
  * One iteration's solver update over all N tokens:
  *   1. v_hat[idx[r]] = v_A[r] for r < M (fresh velocities of A_i);

@@ -68,6 +68,12 @@ def test_device_calls_reject_bad_arguments_on_host(lib):
     assert lib.hsa_select_tokens_pinned(null, null, 8, 2, (C.c_int * 2)(4, 5), null, null, null, 0,
                                         null) == hsa.HSA_EINVAL
     assert lib.hsa_euler_update(null, null, null, null, 0, 8, 6, 0.1, null, null) == hsa.HSA_EINVAL
+    act = (C.c_uint8 * 2)(1, 1)
+    assert lib.hsa_active_rows(null, 8, 2, (C.c_int * 2)(4, 5), act, null, null, null) == hsa.HSA_EINVAL
+    assert lib.hsa_active_rows(null, 8, 0, sizes, act, null, null, null) == hsa.HSA_EINVAL
+    m = C.c_int(-1)
+    assert lib.hsa_active_rows(null, 8, 2, sizes, (C.c_uint8 * 2)(0, 0), null, C.byref(m), null) == hsa.HSA_OK
+    assert m.value == 0                                    # nothing active: no device work
     assert lib.hsa_euler_update(null, null, null, null, 9, 8, 4, 0.1, null, null) == hsa.HSA_EINVAL
     assert lib.hsa_l1_score(null, null, 4, 3, null, null) == hsa.HSA_EINVAL
     assert lib.hsa_layer_step(null, null, null, 8, null, null, null, 1, null, null, null, 0, null, 0,

@@ -100,6 +100,26 @@ def test_select_tokens_pinned_bit_exact(cuda_lib, seed, N, K, kind, pin):
     assert np.array_equal(host(order), want_o)
 
 
+@pytest.mark.parametrize("seed,N,K", [(0, 1000, 3), (1, 32760, 4), (2, 7, 5), (3, 75600, 16)])
+def test_active_rows_bit_exact(cuda_lib, seed, N, K):
+    """A_i from the group lists for every active pattern of K groups (nested or not), against the
+    oracle's active_rows; includes groups of size 0, nothing active and everything active."""
+    r = np.random.default_rng(seed)
+    order = r.permutation(N).astype(np.int32)
+    cuts = np.sort(r.integers(0, N + 1, size=K - 1))
+    sizes = [int(v) for v in np.diff(np.concatenate([[0], cuts, [N]]))]
+    masks = [r.random(K) < 0.5 for _ in range(6)] + [np.zeros(K, bool), np.ones(K, bool)]
+    d_order = torch.from_numpy(order).cuda()
+    for act in masks:
+        idx = torch.full((N + 1,), -9, dtype=torch.int32, device="cuda")
+        M = cuda_lib.active_rows(d_order, sizes, act, idx)
+        want = O.active_rows(order, sizes, act)
+        assert M == len(want)
+        got = host(idx)
+        assert np.array_equal(got[:M], want) and np.all(got[M:] == -9)
+    assert cuda_lib.device_status() == 0
+
+
 # ------------------------------------------------------------------ linear layers
 
 def _lin_case(seed, M, K, Nout, bf16):

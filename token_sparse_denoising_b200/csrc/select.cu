@@ -387,3 +387,52 @@ extern "C" int hsa_select_tokens(const float* d_score, int N, int K, const int* 
                                  int32_t* d_order, void* d_ws, size_t ws_bytes, void* stream) {
   return hsa_select_tokens_pinned(d_score, nullptr, N, K, h_group_sizes, d_group, d_order, d_ws, ws_bytes, stream);
 }
+
+// ------------------------------------------------------------------ A_i from the group lists (§2.1)
+namespace hsa {
+struct RowSegments {
+  int n;                                   // active groups
+  int src[kMaxGroups], dst[kMaxGroups + 1];  // start in order / in A_i; dst[n] = M
+};
+
+// A_i = the active groups' lists of `order`, concatenated in group order.  Grid-stride over the
+// M output positions; each finds its segment among at most 16.
+__global__ void __launch_bounds__(256) k_active_rows(const int32_t* __restrict__ order, RowSegments seg,
+                                                     int32_t* __restrict__ idx) {
+  const int M = seg.dst[seg.n];
+  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < M; r += gridDim.x * blockDim.x) {
+    int k = 0;
+    while (k + 1 < seg.n && r >= seg.dst[k + 1]) ++k;
+    idx[r] = order[seg.src[k] + (r - seg.dst[k])];
+  }
+}
+}  // namespace hsa
+
+extern "C" int hsa_active_rows(const int32_t* d_order, int N, int K, const int* h_group_sizes,
+                               const uint8_t* h_active, int32_t* d_idx, int* h_M, void* stream) {
+  using namespace hsa;
+  if (N < 0 || K < 1 || K > kMaxGroups || !h_group_sizes || !h_active)
+    return set_error(HSA_EINVAL, "active_rows: need N >= 0, 1 <= K <= 16, group sizes and the active mask");
+  RowSegments seg{};
+  long long start = 0;
+  int pos = 0;
+  for (int k = 0; k < K; ++k) {
+    if (h_group_sizes[k] < 0) return set_error(HSA_EINVAL, "active_rows: negative group size");
+    if (h_active[k] && h_group_sizes[k] > 0) {
+      seg.src[seg.n] = (int)start;
+      seg.dst[seg.n] = pos;
+      ++seg.n;
+      pos += h_group_sizes[k];
+    }
+    start += h_group_sizes[k];
+  }
+  if (start != N) return set_error(HSA_EINVAL, "active_rows: group sizes must sum to N");
+  seg.dst[seg.n] = pos;
+  if (h_M) *h_M = pos;
+  if (pos == 0) return HSA_OK;
+  if (!d_order || !d_idx) return set_error(HSA_EINVAL, "active_rows: null device pointer");
+  const int blocks = (pos + 255) / 256 < 4 * num_sms() ? (pos + 255) / 256 : 4 * num_sms();
+  k_active_rows<<<blocks, 256, 0, as_stream(stream)>>>(d_order, seg, d_idx);
+  count_launch(1);
+  return check_launch("active_rows launch");
+}

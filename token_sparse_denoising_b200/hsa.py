@@ -49,6 +49,7 @@ _SIGS = {
     "hsa_select_tokens_workspace_size": (sz, [i32, i32]),
     "hsa_select_tokens": (i32, [vp, i32, i32, vp, vp, vp, vp, sz, vp]),
     "hsa_select_tokens_pinned": (i32, [vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
+    "hsa_active_rows": (i32, [vp, i32, i32, vp, vp, vp, C.POINTER(i32), vp]),
     "hsa_euler_update": (i32, [vp, vp, vp, vp, i32, i32, i32, f32, vp, vp]),
     "hsa_context_kv_workspace_size": (sz, [i32, i32]),
     "hsa_context_kv": (i32, [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -200,6 +201,18 @@ def select_tokens(score, group_sizes, group, order, stream=None, ws=None, pinned
         _check(lib().hsa_select_tokens_pinned(_ptr(score), _ptr(pinned), N, K, sizes.ctypes.data, _ptr(group),
                                               _ptr(order), _ptr(ws), nbytes, _stream(stream)),
                "hsa_select_tokens_pinned")
+
+
+def active_rows(order, group_sizes, active, idx, stream=None) -> int:
+    """A_i: the active groups' lists of `order`, concatenated into `idx`; returns M."""
+    N = order.shape[0]
+    K = len(group_sizes)
+    sizes = np.ascontiguousarray(group_sizes, np.int32)
+    act = np.ascontiguousarray(np.asarray(active, bool).astype(np.uint8))
+    m = C.c_int(0)
+    _check(lib().hsa_active_rows(_ptr(order), N, K, sizes.ctypes.data, act.ctypes.data, _ptr(idx), C.byref(m),
+                                 _stream(stream)), "hsa_active_rows")
+    return int(m.value)
 
 
 def euler_update(x, vhat, vA, idx, dsigma: float, score=None, stream=None):

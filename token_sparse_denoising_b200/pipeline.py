@@ -179,12 +179,7 @@ class HSARun:
         first_off = next((k for k in range(K) if not act[k]), K)
         if not act[first_off:].any():
             return self.order[:M]            # nested budgets: the active groups are a prefix
-        pos = 0
-        for k in range(K):
-            if act[k] and self.sizes[k]:
-                n = self.sizes[k]
-                self.idx_buf[pos:pos + n].copy_(self.order[self.starts[k]:self.starts[k] + n])
-                pos += n
+        hsa.active_rows(self.order, self.sizes, act, self.idx_buf)
         return self.idx_buf[:M]
 
     def step(self, record: list | None = None):
