@@ -161,6 +161,8 @@ class Step:
         self.score = torch.zeros(N, device=device)
         self.group = torch.zeros(N, dtype=torch.int8, device=device)
         self.order = torch.arange(N, dtype=torch.int32, device=device)
+        self.sel_ws = torch.empty(max(hsa.select_tokens_workspace_size(N, len(self.sizes)), 1), dtype=torch.uint8,
+                                  device=device)
         # active sets of the sweep: top-M tokens by the L1 score of two velocity draws
         va, vb = torch.from_numpy(inp["va"]).to(device), torch.from_numpy(inp["vb"]).to(device)
         s = torch.empty(N, device=device)
@@ -181,7 +183,7 @@ class Step:
         idx = self.order
         vA = self.model.velocity(self.x, idx)
         hsa.euler_update(self.x, self.vhat, vA, idx, DSIGMA, score=self.score)
-        hsa.select_tokens(self.score, self.sizes, self.group, self.order)
+        hsa.select_tokens(self.score, self.sizes, self.group, self.order, ws=self.sel_ws)
 
     def partial(self, f):
         """One iteration of the cached window: the layer step on the top-M set, then cached Euler."""
