@@ -13,9 +13,11 @@
 // One 1024-thread CTA (the work is a few passes over N floats):
 //   1. for each boundary c_k (k < K): radix-select, over the 32-bit order key,
 //      the element of rank c_k - 1 (4 passes of 8 bits; per-warp private
-//      shared-memory histograms, since scores share few exponent bytes; the
-//      top-digit pass is shared by all boundaries), then the right index among
-//      the equal keys by a block scan;
+//      shared-memory histograms, since scores share few exponent bytes).  The
+//      top-digit pass is shared by all boundaries, and each later pass serves
+//      two boundaries at once: their key subsets are disjoint or identical, so
+//      one sweep fills both histograms.  Then the right index among the equal
+//      keys by a block scan;
 //   2. each token's group = number of boundaries it ranks at or after;
 //   3. the groups' lists, each ascending by index: warp w owns a contiguous index
 //      range and walks it 32 consecutive indices at a time (bank-conflict-free
@@ -32,9 +34,9 @@ namespace hsa {
 constexpr int kSelectThreads = 1024;
 constexpr int kMaxGroups = 16;
 
-// Largest N whose keys are staged in shared memory (4 bytes each, on top of ~35 KB of
+// Largest N whose keys are staged in shared memory (4 bytes each, on top of ~70 KB of
 // histograms); larger N reads the scores from global memory on every pass.
-constexpr int kSelectStagedMax = 40960;
+constexpr int kSelectStagedMax = 36864;
 
 struct SelectArgs {
   int K;
@@ -98,75 +100,97 @@ struct KeySource {
   }
 };
 
-__device__ void radix_pass(KeySource key, int N, uint32_t mask, uint32_t prefix, int shift,
-                           int rank, uint32_t (*hw)[257], uint32_t* hist, int* out_digit, int* out_rank) {
+constexpr int kHistStride = 513;   // per-warp histogram row: 2 x 256 bins, odd stride
+
+// One warp finds, in bins[0, 256), the digit holding the element of rank `rank` and the rank within
+// it: lane l owns bins [8l, 8l+8) (local sums, warp exclusive scan, the owning lane walks its bins).
+__device__ __forceinline__ void scan_bins(const uint32_t* bins, int rank, int* out_digit, int* out_rank) {
+  const int lane = threadIdx.x & 31;
+  uint32_t v[8], s = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    v[e] = bins[8 * lane + e];
+    s += v[e];
+  }
+  uint32_t incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint32_t excl = incl - s;
+  if ((uint32_t)rank >= excl && (uint32_t)rank < incl) {
+    uint32_t r = (uint32_t)rank - excl;
+    int d = 0;
+    for (; d < 7; ++d) {
+      if (r < v[d]) break;
+      r -= v[d];
+    }
+    *out_digit = 8 * lane + d;
+    *out_rank = (int)r;
+  }
+}
+
+// One radix pass for nt <= 2 targets t, each a (prefix, mask) of the keys already fixed and the rank
+// sought among them: the histogram of the 8-bit digit at `shift` of every target's keys (per-warp
+// private copies, then summed), then, by warp t, target t's digit and the rank within that digit.
+// Two targets select either disjoint key sets (different prefixes: bins [0,256) and [256,512)) or the
+// same one (equal prefix and mask: both read bins [0,256)), so one sweep over the keys serves both.
+// Every thread of the block calls it; hist keeps the summed bins for the caller.
+__device__ void radix_pass2(KeySource key, int N, int nt, const uint32_t* prefix, const uint32_t* mask,
+                            const int* rank, int shift, uint32_t (*hw)[kHistStride], uint32_t* hist,
+                            int* out_digit, int* out_rank) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = lane; i < 257; i += 32) hw[warp][i] = 0;
+  const bool shared_keys = nt == 2 && prefix[0] == prefix[1] && mask[0] == mask[1];
+  const bool two = nt == 2 && !shared_keys;
+  const int nbins = two ? 512 : 256;
+  const uint32_t p0 = prefix[0], m0 = mask[0];
+  const uint32_t p1 = two ? prefix[1] : 0u, m1 = two ? mask[1] : 0u;
+  for (int i = lane; i < nbins; i += 32) hw[warp][i] = 0;
   __syncwarp();
   // Keys of similar scores share their top bytes, so most lanes of a warp often carry the
-  // same digit: the lanes equal to lane 0's digit add with one atomic, the rest one each.
+  // same bin: the lanes equal to lane 0's bin add with one atomic, the rest one each.
   for (int base = 0; base < N; base += kSelectThreads) {
     const int n = base + tid;
-    uint32_t digit = 0xFFFFu;                       // no contribution
+    uint32_t bin = 0xFFFFu;                         // no contribution
     if (n < N) {
       const uint32_t ik = key(n);
-      if ((ik & mask) == prefix) digit = (ik >> shift) & 255u;
+      if ((ik & m0) == p0) bin = (ik >> shift) & 255u;
+      else if (two && (ik & m1) == p1) bin = 256u + ((ik >> shift) & 255u);
     }
-    const uint32_t lead = __shfl_sync(0xffffffffu, digit, 0);
-    const unsigned same = __ballot_sync(0xffffffffu, digit == lead);
+    const uint32_t lead = __shfl_sync(0xffffffffu, bin, 0);
+    const unsigned same = __ballot_sync(0xffffffffu, bin == lead);
     if (lane == 0 && lead != 0xFFFFu) atomicAdd(&hw[warp][lead], (uint32_t)__popc(same));
-    if (digit != lead && digit != 0xFFFFu) atomicAdd(&hw[warp][digit], 1u);
+    if (bin != lead && bin != 0xFFFFu) atomicAdd(&hw[warp][bin], 1u);
   }
   __syncthreads();
-  if (tid < 256) {
+  if (tid < nbins) {
     uint32_t t = 0;
 #pragma unroll 8
     for (int w = 0; w < kSelectThreads / 32; ++w) t += hw[w][tid];
     hist[tid] = t;
   }
   __syncthreads();
-  if (warp == 0) {
-    // lane l owns bins [8l, 8l+8): local sums, warp exclusive scan, then the lane whose
-    // range holds `rank` walks its 8 bins
-    uint32_t v[8], s = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      v[e] = hist[8 * lane + e];
-      s += v[e];
-    }
-    uint32_t incl = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const uint32_t excl = incl - s;
-    if ((uint32_t)rank >= excl && (uint32_t)rank < incl) {
-      uint32_t r = (uint32_t)rank - excl;
-      int d = 0;
-      for (; d < 7; ++d) {
-        if (r < v[d]) break;
-        r -= v[d];
-      }
-      *out_digit = 8 * lane + d;
-      *out_rank = (int)r;
-    }
-  }
+  if (warp < nt) scan_bins(hist + (two && warp == 1 ? 256 : 0), rank[warp], out_digit + warp, out_rank + warp);
   __syncthreads();
 }
 
 __global__ void __launch_bounds__(kSelectThreads, 1)
     k_select(const float* __restrict__ score, const uint8_t* __restrict__ pinned, int N, SelectArgs a,
              int8_t* __restrict__ group, int* __restrict__ order) {
-  __shared__ uint32_t hw[kSelectThreads / 32][257];   // per-warp private histograms
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t hist0[256];                      // first-pass histogram, shared by all boundaries
+  __shared__ uint32_t hist[512];
   __shared__ int warp_sums[33];
   __shared__ int s_wcnt[kMaxGroups][kSelectThreads / 32];   // per group, per warp: count, then offset
   __shared__ uint32_t s_thr_key[kMaxGroups];
   __shared__ int s_thr_idx[kMaxGroups];
-  __shared__ int s_digit, s_rank;
-  extern __shared__ uint32_t s_ikeys[];                // N staged keys when the launch provides them
+  __shared__ uint32_t s_pref[kMaxGroups], s_mask[kMaxGroups];   // per inner boundary (compacted list)
+  __shared__ int s_rank[kMaxGroups], s_bnd[kMaxGroups];
+  __shared__ int s_digit2[2], s_rank2[2];
+  // dynamic shared memory: the per-warp private histograms, then the N staged keys when the launch
+  // provides them
+  extern __shared__ uint32_t s_dyn[];
+  uint32_t (*hw)[kHistStride] = reinterpret_cast<uint32_t (*)[kHistStride]>(s_dyn);
+  uint32_t* s_ikeys = s_dyn + (kSelectThreads / 32) * kHistStride;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int kWarps = kSelectThreads / 32;
@@ -181,95 +205,93 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
     key.ikeys = s_ikeys;
   }
 
-  // ---- 1. threshold element of every inner boundary
-  bool first_done = false;
+  // ---- 1. threshold element of every inner boundary.  Ascending order of ik = ~key is descending
+  // score order; boundary c_b needs the element of rank c_b - 1.  Boundaries with c_b <= 0 or
+  // c_b >= N need no threshold.
+  int nb = 0;
   for (int b = 1; b < a.K; ++b) {
     const int c = a.cum[b];
-    if (c <= 0 || c >= N) continue;  // empty prefix or everything: no threshold needed
-    // ascending order of ik = ~key is descending score order; find the element of rank c - 1
-    uint32_t prefix = 0, mask = 0;
-    int rank = c - 1;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      if (shift == 24 && first_done) {
-        // the top-digit histogram does not depend on the boundary: reuse it
-        if (tid < 256) hist[tid] = hist0[tid];
-        __syncthreads();
-        if (tid < 32) {
-          uint32_t v[8], sum = 0;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            v[e] = hist[8 * tid + e];
-            sum += v[e];
-          }
-          uint32_t incl = sum;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (tid >= o) incl += y;
-          }
-          const uint32_t excl = incl - sum;
-          if ((uint32_t)rank >= excl && (uint32_t)rank < incl) {
-            uint32_t r = (uint32_t)rank - excl;
-            int d = 0;
-            for (; d < 7; ++d) {
-              if (r < v[d]) break;
-              r -= v[d];
-            }
-            s_digit = 8 * tid + d;
-            s_rank = (int)r;
-          }
-        }
-        __syncthreads();
-      } else {
-        radix_pass(key, N, mask, prefix, shift, rank, hw, hist, &s_digit, &s_rank);
-        if (shift == 24) {
-          if (tid < 256) hist0[tid] = hist[tid];
-          first_done = true;
-        }
+    if (c > 0 && c < N) {
+      if (tid == 0) {
+        s_bnd[nb] = b;
+        s_rank[nb] = c - 1;
+        s_pref[nb] = 0u;
+        s_mask[nb] = 0u;
       }
-      prefix |= (uint32_t)s_digit << shift;
-      mask |= 255u << shift;
-      rank = s_rank;
+      ++nb;
+    }
+  }
+  __syncthreads();
+  if (nb > 0) {
+    // top byte: one histogram serves every boundary
+    radix_pass2(key, N, 1, s_pref, s_mask, s_rank, 24, hw, hist, s_digit2, s_rank2);
+    if (warp == 0) {
+      for (int i = 0; i < nb; ++i) {
+        scan_bins(hist, s_rank[i], s_digit2, s_rank2);
+        __syncwarp();
+        if (lane == 0) {
+          s_pref[i] = (uint32_t)s_digit2[0] << 24;
+          s_mask[i] = 255u << 24;
+          s_rank[i] = s_rank2[0];
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+  }
+  for (int i0 = 0; i0 < nb; i0 += 2) {
+    const int nt = nb - i0 < 2 ? nb - i0 : 2;
+    for (int shift = 16; shift >= 0; shift -= 8) {
+      radix_pass2(key, N, nt, s_pref + i0, s_mask + i0, s_rank + i0, shift, hw, hist, s_digit2, s_rank2);
+      if (tid < nt) {
+        s_pref[i0 + tid] |= (uint32_t)s_digit2[tid] << shift;
+        s_mask[i0 + tid] |= 255u << shift;
+        s_rank[i0 + tid] = s_rank2[tid];
+      }
       __syncthreads();
     }
-    // the rank-th smallest token index among keys equal to the target: per-warp counts of
-    // matches, a scan over the warps, then the warp holding that rank finds the lane
-    int cnt = 0;
-    for (int base = wlo; base < whi; base += 32) {
-      const int n = base + lane;
-      cnt += __popc(__ballot_sync(0xffffffffu, n < whi && key(n) == prefix));
-    }
-    if (lane == 0) warp_sums[warp] = cnt;
-    __syncthreads();
-    if (warp == 0) {
-      const int v = warp_sums[lane];
-      int incl = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      warp_sums[lane] = incl - v;
-    }
-    __syncthreads();
-    const int excl = warp_sums[warp];
-    if (rank >= excl && rank < excl + cnt) {      // warp-uniform
-      int seen = excl;
+    for (int t = 0; t < nt; ++t) {
+      const uint32_t prefix = s_pref[i0 + t];
+      const int rank = s_rank[i0 + t], b = s_bnd[i0 + t];
+      // the rank-th smallest token index among keys equal to the target: per-warp counts of
+      // matches, a scan over the warps, then the warp holding that rank finds the lane
+      int cnt = 0;
       for (int base = wlo; base < whi; base += 32) {
         const int n = base + lane;
-        const bool m = n < whi && key(n) == prefix;
-        const unsigned mk = __ballot_sync(0xffffffffu, m);
-        if (rank < seen + __popc(mk)) {
-          if (m && seen + __popc(mk & lanes_below) == rank) {
-            s_thr_idx[b] = n;
-            s_thr_key[b] = ~prefix;
-          }
-          break;
-        }
-        seen += __popc(mk);
+        cnt += __popc(__ballot_sync(0xffffffffu, n < whi && key(n) == prefix));
       }
+      if (lane == 0) warp_sums[warp] = cnt;
+      __syncthreads();
+      if (warp == 0) {
+        const int v = warp_sums[lane];
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        warp_sums[lane] = incl - v;
+      }
+      __syncthreads();
+      const int excl = warp_sums[warp];
+      if (rank >= excl && rank < excl + cnt) {      // warp-uniform
+        int seen = excl;
+        for (int base = wlo; base < whi; base += 32) {
+          const int n = base + lane;
+          const bool m = n < whi && key(n) == prefix;
+          const unsigned mk = __ballot_sync(0xffffffffu, m);
+          if (rank < seen + __popc(mk)) {
+            if (m && seen + __popc(mk & lanes_below) == rank) {
+              s_thr_idx[b] = n;
+              s_thr_key[b] = ~prefix;
+            }
+            break;
+          }
+          seen += __popc(mk);
+        }
+      }
+      __syncthreads();
     }
-    __syncthreads();
   }
 
   // ---- 2. group of each token; per-warp counts per group.  Loops over groups are unrolled to
@@ -367,13 +389,14 @@ extern "C" int hsa_select_tokens_pinned(const float* d_score, const uint8_t* d_p
   if (c != N) return set_error(HSA_EINVAL, "select: group sizes must sum to N");
   if (N == 0) return HSA_OK;
   a.staged = N <= kSelectStagedMax ? 1 : 0;
-  const size_t dyn = a.staged ? (size_t)N * sizeof(uint32_t) : 0;
+  constexpr size_t kHistBytes = (size_t)(kSelectThreads / 32) * kHistStride * sizeof(uint32_t);
+  const size_t dyn = kHistBytes + (a.staged ? (size_t)N * sizeof(uint32_t) : 0);
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
     if (cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSelectStagedMax * (int)sizeof(uint32_t)) != cudaSuccess)
+                             (int)kHistBytes + kSelectStagedMax * (int)sizeof(uint32_t)) != cudaSuccess)
       return check_launch("select: shared-memory attribute");
     attr_done[dev] = true;
   }
