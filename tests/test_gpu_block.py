@@ -61,6 +61,51 @@ def test_layer_step_bf16_small(cuda_lib, cross, frac):
     assert np.array_equal(kc[skipped], Kc0[skipped]) and np.array_equal(vc[skipped], Vc0[skipped])
 
 
+@pytest.mark.parametrize("bf16,cross", [(True, False), (True, True), (False, False)])
+def test_layer_step_single_token(cuda_lib, bf16, cross):
+    """Degenerate case: one token (N = M = 1), so attention has a single key and every tile is ragged."""
+    grid = S.Grid(1, 1, 1)
+    shape, bw = _block(21, 256, 512, cross, bf16)
+    idx = np.array([0], np.int32)
+    x = S.normal(22, (1, 256))
+    Kc0, Vc0 = S.normal(23, (1, 256), 1.0, bf16), S.normal(24, (1, 256), 1.0, bf16)
+    ctx = S.normal(25, (16, 256), 1.0, bf16) if cross else None
+    xA, kc, vc, _ = _run_layer_step(bw, bf16, grid, idx, x, Kc0, Vc0, ctx)
+    want, Kw, Vw = O.dit_block_active(bw, x, idx, S.token_positions(grid), Kc0, Vc0,
+                                      O.context_kv(bw, ctx) if cross else None)
+    close = assert_bf16_close if bf16 else assert_f32_close
+    close(xA - x, want - x, "block output delta")
+    close(kc, Kw, "K cache")
+
+
+def test_layer_step_with_spare_workspace_splits_attention(cuda_lib):
+    """A workspace sized for every token, used with a small active set, lets the attention split its
+    incomplete last wave over key ranges (N = 2000 keys, M = 100: two heads' units, each split); the
+    result matches the oracle like the unsplit path."""
+    grid = S.Grid(5, 20, 20)
+    N = grid.N
+    shape, bw = _block(31, 256, 512, True, True)
+    M = 100
+    idx = S.scattered_mask(32, N, M)
+    x = S.normal(33, (N, 256))
+    Kc0, Vc0 = S.normal(34, (N, 256), 1.0, True), S.normal(35, (N, 256), 1.0, True)
+    ctx = S.normal(36, (16, 256), 1.0, True)
+    assert hsa.attention_workspace_size(M, N, 2, hsa.HSA_BF16) > 0           # this shape does split
+    w = hsa.LayerWeights(bw, "cuda", True)
+    kc, vc = dev(Kc0, torch.bfloat16), dev(Vc0, torch.bfloat16)
+    xA = torch.empty((M, 256), device="cuda")
+    ws = torch.empty(hsa.layer_step_workspace_size(N, 256, 512, w.dtype), dtype=torch.uint8, device="cuda")
+    ck = torch.empty((16, 256), dtype=torch.bfloat16, device="cuda")
+    cv = torch.empty_like(ck)
+    cws = torch.empty(hsa.context_kv_workspace_size(16, 256), dtype=torch.uint8, device="cuda")
+    hsa.context_kv(dev(ctx, torch.bfloat16), w.t["w_kv2"], w.t["b_kv2"], w.t["g_k2"], ck, cv, cws)
+    hsa.layer_step(w, kc, vc, xA, dev(idx), dev(S.token_positions(grid)), ws, x_src=dev(x), ctx_k=ck, ctx_v=cv)
+    assert hsa.device_status() == 0
+    want, Kw, _ = O.dit_block_active(bw, x[idx], idx, S.token_positions(grid), Kc0, Vc0, O.context_kv(bw, ctx))
+    assert_bf16_close(host(xA) - x[idx], want - x[idx], "block output delta")
+    assert_bf16_close(host(kc)[idx], Kw[idx], "fresh K rows")
+
+
 def test_layer_step_f32_tiny_shape(cuda_lib):
     wl = S.TINY_FP32
     grid = wl.grid
