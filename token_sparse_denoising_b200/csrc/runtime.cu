@@ -1,5 +1,6 @@
 // runtime.cu -- host side of libhsa: error text, the device status word, launch
-// counting and TMA tensor-map encoding.
+// counting, per-class kernel timing and TMA tensor-map encoding; plus the one-warp
+// kernel behind hsa_selftest_wait_timeout, which checks the bounded-wait failure path.
 #include <cudaTypedefs.h>
 
 #include <atomic>

@@ -25,8 +25,11 @@
 //      ballots, one scan over the warps per group gives each warp its offsets,
 //      and a lane's position is the number of lower lanes in its group.  Group k
 //      starts at c_{k-1}.
-// For N <= 40960 the order keys are first staged in shared memory, so the passes
+// For N <= 36864 the order keys are first staged in shared memory, so the passes
 // do not wait on L2 latency for every element.
+//
+// Also here: k_active_rows, which builds A_i from the group lists when the active
+// groups are not a prefix of the order (non-nested budgets).
 #include "common.cuh"
 
 namespace hsa {
