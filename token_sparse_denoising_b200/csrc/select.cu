@@ -139,13 +139,16 @@ __device__ __forceinline__ void scan_bins(const uint32_t* bins, int rank, int* o
 // private copies, then summed), then, by warp t, target t's digit and the rank within that digit.
 // Two targets select either disjoint key sets (different prefixes: bins [0,256) and [256,512)) or the
 // same one (equal prefix and mask: both read bins [0,256)), so one sweep over the keys serves both.
-// Every thread of the block calls it; hist keeps the summed bins for the caller.
-__device__ void radix_pass2(KeySource key, int N, int nt, const uint32_t* prefix, const uint32_t* mask,
+// Every thread of the block calls it; hist keeps the summed bins for the caller.  NT is a template
+// parameter so the single-target pass carries no second-target test per key.
+template <int NT>
+__device__ void radix_pass2(KeySource key, int N, const uint32_t* prefix, const uint32_t* mask,
                             const int* rank, int shift, uint32_t (*hw)[kHistStride], uint32_t* hist,
                             int* out_digit, int* out_rank) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool shared_keys = nt == 2 && prefix[0] == prefix[1] && mask[0] == mask[1];
-  const bool two = nt == 2 && !shared_keys;
+  constexpr int nt = NT;
+  const bool shared_keys = NT == 2 && prefix[0] == prefix[1] && mask[0] == mask[1];
+  const bool two = NT == 2 && !shared_keys;
   const int nbins = two ? 512 : 256;
   const uint32_t p0 = prefix[0], m0 = mask[0];
   const uint32_t p1 = two ? prefix[1] : 0u, m1 = two ? mask[1] : 0u;
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
   __syncthreads();
   if (nb > 0) {
     // top byte: one histogram serves every boundary
-    radix_pass2(key, N, 1, s_pref, s_mask, s_rank, 24, hw, hist, s_digit2, s_rank2);
+    radix_pass2<1>(key, N, s_pref, s_mask, s_rank, 24, hw, hist, s_digit2, s_rank2);
     if (warp == 0) {
       for (int i = 0; i < nb; ++i) {
         scan_bins(hist, s_rank[i], s_digit2, s_rank2);
@@ -245,7 +248,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
   for (int i0 = 0; i0 < nb; i0 += 2) {
     const int nt = nb - i0 < 2 ? nb - i0 : 2;
     for (int shift = 16; shift >= 0; shift -= 8) {
-      radix_pass2(key, N, nt, s_pref + i0, s_mask + i0, s_rank + i0, shift, hw, hist, s_digit2, s_rank2);
+      if (nt == 2)
+        radix_pass2<2>(key, N, s_pref + i0, s_mask + i0, s_rank + i0, shift, hw, hist, s_digit2, s_rank2);
+      else
+        radix_pass2<1>(key, N, s_pref + i0, s_mask + i0, s_rank + i0, shift, hw, hist, s_digit2, s_rank2);
       if (tid < nt) {
         s_pref[i0 + tid] |= (uint32_t)s_digit2[tid] << shift;
         s_mask[i0 + tid] |= 255u << shift;
