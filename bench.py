@@ -546,8 +546,11 @@ def run_wan14(args):
 
 # ---------------------------------------------------------------- the oracle on the host cores
 
-ORACLE_ROWS = 32        # attention / O / cross / FFN query rows per sample
-ORACLE_PROJ = 4096      # tokens whose q/k/v projections, Euler update and score run per sample
+# (tokens whose q/k/v projections, Euler update and score run; query rows whose attention, O-projection,
+# cross-attention and FFN run) per sample: ~10 s of host work for the baseline beside the GPU numbers,
+# ~1 s per step for the reference arm, whose whole run must end within minutes.
+BASELINE_SAMPLE = (32760, 512)
+REFERENCE_SAMPLE = (4096, 32)
 
 
 def blas_threads() -> int:
@@ -561,21 +564,23 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def oracle_step_sample(inp):
+def oracle_step_sample(inp, sample):
     """Time the oracle on a bounded sample of one full iteration; return the extrapolated ms per step.
 
     Every part of the step is linear in the rows it touches, so each is timed on
-    a spread sample and scaled: the q/k/v projections (LN, GEMM, RMSNorm, RoPE)
-    and the cached Euler update + L1 score of ORACLE_PROJ tokens (x N/4096);
-    attention over all N cache rows + O-projection + cross-attention + FFN of
-    ORACLE_ROWS query rows (x N/32); the regrouping runs on all N scores.
+    a spread sample and scaled. `sample` = (n_proj, n_rows): the q/k/v projections
+    (LN, GEMM, RMSNorm, RoPE) and the cached Euler update + L1 score of n_proj
+    tokens (x N/n_proj); attention over all N cache rows + O-projection +
+    cross-attention + FFN of n_rows query rows (x N/n_rows); the regrouping runs
+    on all N scores.
     """
     from oracle import hsa_oracle as O
     N = GRID.N
+    n_proj, n_rows = min(sample[0], N), min(sample[1], sample[0], N)
     bw, pos = inp["bw"], inp["pos"]
     ctx_kv = O.context_kv(bw, inp["ctx"])            # once per run: not part of a step
-    proj = np.arange(0, N, N // ORACLE_PROJ)[:ORACLE_PROJ]
-    qrows = np.arange(0, ORACLE_PROJ, ORACLE_PROJ // ORACLE_ROWS)[:ORACLE_ROWS]
+    proj = np.arange(0, N, N // n_proj)[:n_proj]
+    qrows = np.arange(0, n_proj, n_proj // n_rows)[:n_rows]
     X = inp["x0"][proj].astype(np.float64)
     Kc, Vc = inp["kc0"].astype(np.float64), inp["vc0"].astype(np.float64)
     t0 = time.perf_counter()
@@ -600,7 +605,7 @@ def oracle_step_sample(inp):
 
 
 def cpu_baseline(inp):
-    est_ms, wall, sample = oracle_step_sample(inp)
+    est_ms, wall, sample = oracle_step_sample(inp, BASELINE_SAMPLE)
     return {"value": round(est_ms, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
             "sample": sample, "wall_s": round(wall, 2)}
 
@@ -608,10 +613,10 @@ def cpu_baseline(inp):
 def run_reference(args):
     inp = synthetic_inputs()
     for _ in range(args.warmup):
-        oracle_step_sample(inp)
+        oracle_step_sample(inp, REFERENCE_SAMPLE)
     vals, wall, sample = [], 0.0, ""
     for _ in range(args.steps):
-        v, w, sample = oracle_step_sample(inp)
+        v, w, sample = oracle_step_sample(inp, REFERENCE_SAMPLE)
         vals.append(v)
         wall += w
     value = float(np.mean(vals))
