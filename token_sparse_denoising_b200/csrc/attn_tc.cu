@@ -12,7 +12,8 @@
 //   warp 1      TMEM owner (512 columns) and MMA issuer (the warp runs the loop with
 //               warp-uniform descriptors, one elected lane issues):
 //                 S_b = Q K_j^T          (SS: both K-major, 128 x 128 x 128), b = j % 2
-//                 O_b += P_j V_j         (TS: P from TMEM, V MN-major)
+//                 O_b += P_j V_j         (TS: P from TMEM, V MN-major), in two halves of
+//                                        64 keys, each issued as soon as its P is stored
 //               QK^T of tile j+2 is issued right after PV of tile j, so the tensor
 //               pipe alternates between the two parities.
 //   warps 2..9  softmax, one thread per query row and all 128 key columns of a tile:
@@ -21,7 +22,8 @@
 //               and O accumulator, so the two warps of a sub-partition never wait for
 //               each other and one's exponentials overlap the other's loads, max and
 //               stores.  p = 2^(t - m) goes back to TMEM as bf16 over the first 64
-//               columns of the S buffer it came from.  O_b is rescaled in TMEM only
+//               columns of the S buffer it came from; the first 32 columns (keys 0-63)
+//               are released to the MMA warp before the second half's exponentials end.  O_b is rescaled in TMEM only
 //               when the max grew by more than 2^8 (the stale max keeps p <= 256).
 //               The epilogue merges the two parities: O = (a0 O_0 + a1 O_1) / (a0 l_0
 //               + a1 l_1) with a_b = 2^(m_b - max(m_0, m_1)).
@@ -61,7 +63,7 @@ struct AttnShared {
   uint64_t q_full;
   uint64_t k_full[kKSlots], k_empty[kKSlots];
   uint64_t v_full[kVSlots], v_empty[kVSlots];
-  uint64_t s_full[2], p_full[2], o_done;
+  uint64_t s_full[2], p_full[2][2], o_done;   // p_full[parity][half]: P of keys [64 h, 64 h + 64) stored
   uint32_t tmem;
   float xm[2][128], xl[2][128];  // [parity][row]: running max and sum, merged in the epilogue
 };
@@ -165,7 +167,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->s_full[b], 1);
-      mbar_init(&sh->p_full[b], 128);
+      mbar_init(&sh->p_full[b][0], 128);
+      mbar_init(&sh->p_full[b][1], 128);
     }
     mbar_init(&sh->o_done, 1);
     fence_mbar_init();
@@ -256,20 +259,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (ok && nj > 1) ok = issue_qk(1);
     for (int j = 0; ok && j < nj; ++j) {
       const int b = j & 1, sv = j % kVSlots;
-      if (!wait_all(&sh->p_full[b], (j >> 1) & 1)) break;
-      if (!wait_all(&sh->v_full[sv], (j / kVSlots) & 1)) break;
-      tc_fence_after();
       const uint64_t vd = v_desc + (uint64_t)((sv * kTileBytes) >> 4);
-      if (leader) {
+      // PV in two halves of 64 keys: the first half starts while the softmax warps are still
+      // computing the exponentials of the second
+      bool got = true;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // V tile: key rows of 128 B (64 channels) per box; 16 keys = two 1024-byte atoms
-          umma_ts(tm + kColO + b * 128, tm + kColS + b * 128 + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), idesc_o,
-                  (j >= 2 || kk > 0));
+      for (int half = 0; half < 2; ++half) {
+        if (!wait_all(&sh->p_full[b][half], (j >> 1) & 1)) { got = false; break; }
+        if (half == 0 && !wait_all(&sh->v_full[sv], (j / kVSlots) & 1)) { got = false; break; }
+        tc_fence_after();
+        if (leader) {
+#pragma unroll
+          for (int kk = half * 4; kk < half * 4 + 4; ++kk) {
+            // V tile: key rows of 128 B (64 channels) per box; 16 keys = two 1024-byte atoms
+            umma_ts(tm + kColO + b * 128, tm + kColS + b * 128 + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), idesc_o,
+                    (j >= 2 || kk > 0));
+          }
+          if (half == 1) umma_commit(&sh->v_empty[sv]);
         }
-        umma_commit(&sh->v_empty[sv]);
+        __syncwarp();
       }
-      __syncwarp();
+      if (!got) break;
       if (j + 2 < nj) ok = issue_qk(j + 2);   // overwrites S_b (P_j) after PV_j in issue order
     }
     if (leader) umma_commit(&sh->o_done);   // every MMA of this CTA, both O accumulators
@@ -319,6 +329,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         l *= corr;
         m = m_tile;
       }
+      // a warp that rescales O_par releases both halves of P after the rescale; the others
+      // release the first half as soon as it is stored
+      const bool any_need = __any_sync(0xffffffffu, need);
       const float neg_m = -m;
       const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(neg_m, neg_m);
       float2 rs4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -333,15 +346,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const float p1 = poly ? ex2_poly(x.y) : ex2_approx(x.y);
           rs4[(c >> 1) & 3] = fadd2(rs4[(c >> 1) & 3], make_float2(p0, p1));
           pk[(c >> 1) & 31] = pack_bf16x2(p0, p1);
+          if (c == 64 + 14 && !any_need) {
+            // the first half's store has had eight column pairs of exponentials to land
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sh->p_full[par][0]);
+          }
         }
         // P column i holds keys 2i, 2i+1 of the tile, over S_par's first 64 columns
         tmem_st32(s_col + hh * 32, pk);
       }
       l += ((rs4[0].x + rs4[0].y) + (rs4[1].x + rs4[1].y)) + ((rs4[2].x + rs4[2].y) + (rs4[3].x + rs4[3].y));
-      if (__any_sync(0xffffffffu, need)) {
+      if (any_need) {
         // O_par holds PV of this parity's previous tile, complete: S_par was written by an MMA
         // issued after that PV, and the s_full wait above covered it.  PV of this tile starts
-        // only after the p_full arrival below.
+        // only after this warp's p_full arrivals below.
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
@@ -354,7 +373,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&sh->p_full[par]);
+      if (any_need) mbar_arrive(&sh->p_full[par][0]);
+      mbar_arrive(&sh->p_full[par][1]);
     }
     // ---------------------------------------------------------------- epilogue
     // merge the two parities; parity 1 has tiles only when nj >= 2
