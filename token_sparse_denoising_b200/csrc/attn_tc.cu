@@ -65,9 +65,12 @@ constexpr int kPolyPer8 = HSA_ATTN_POLY_PER8;
 
 struct AttnShared {
   uint64_t q_full;
-  uint64_t k_full[kKSlots], k_empty[kKSlots];
-  uint64_t v_full[kVSlots], v_empty[kVSlots];
-  uint64_t s_full[2], p_full[2][2], o_done;   // p_full[parity][half]: P of keys [64 h, 64 h + 64) stored
+  uint64_t k_full[2], k_empty[kKSlots];    // k_full: tiles 0 and 1 only
+  uint64_t v_empty[kVSlots];
+  // p_full[b][h]: P of keys [64 h, 64 h + 64) of tile j (b = j % 2) stored by the 128 softmax
+  // threads, plus one producer arrival with the bytes of the next operand the MMA warp needs:
+  // V_j for h = 0, K_{j+2} for h = 1 (a plain arrival when there is no tile j+2)
+  uint64_t s_full[2], p_full[2][2], o_done;
   uint32_t tmem;
   float xm[2][128], xl[2][128];  // [parity][row]: running max and sum, merged in the epilogue
 };
@@ -161,18 +164,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&sh->q_full, 1);
-    for (int s = 0; s < kKSlots; ++s) {
-      mbar_init(&sh->k_full[s], 1);
-      mbar_init(&sh->k_empty[s], 1);
-    }
-    for (int s = 0; s < kVSlots; ++s) {
-      mbar_init(&sh->v_full[s], 1);
-      mbar_init(&sh->v_empty[s], 1);
-    }
+    for (int s = 0; s < kKSlots; ++s) mbar_init(&sh->k_empty[s], 1);
+    for (int s = 0; s < 2; ++s) mbar_init(&sh->k_full[s], 1);
+    for (int s = 0; s < kVSlots; ++s) mbar_init(&sh->v_empty[s], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->s_full[b], 1);
-      mbar_init(&sh->p_full[b][0], 128);
-      mbar_init(&sh->p_full[b][1], 128);
+      mbar_init(&sh->p_full[b][0], 129);
+      mbar_init(&sh->p_full[b][1], 129);
     }
     mbar_init(&sh->o_done, 1);
     fence_mbar_init();
@@ -198,32 +196,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tma_load_2d(sQ, &tmQ, &sh->q_full, x0, m0);
       tma_load_2d(sQ + kTileBytes / 2, &tmQ, &sh->q_full, x0 + 64, m0);
     }
-    auto load_k = [&](int j) -> bool {
+    // K_j into its ring slot, completing on `bar`
+    auto load_k = [&](int j, uint64_t* bar) -> bool {
       const int sk = j % kKSlots;
       const bool ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->k_empty[sk], ((j / kKSlots) & 1) ^ 1), 0);
       __syncwarp();
       if (ok && leader) {
         uint8_t* k = sK + sk * kTileBytes;
-        mbar_expect_tx(&sh->k_full[sk], kTileBytes);
-        tma_load_2d(k, &tmK, &sh->k_full[sk], x0, (j0 + j) * kAttnBN);
-        tma_load_2d(k + kTileBytes / 2, &tmK, &sh->k_full[sk], x0 + 64, (j0 + j) * kAttnBN);
+        mbar_expect_tx(bar, kTileBytes);
+        tma_load_2d(k, &tmK, bar, x0, (j0 + j) * kAttnBN);
+        tma_load_2d(k + kTileBytes / 2, &tmK, bar, x0 + 64, (j0 + j) * kAttnBN);
       }
       return ok;
     };
-    bool ok = load_k(0);
-    if (ok && nj > 1) ok = load_k(1);
+    bool ok = load_k(0, &sh->k_full[0]);
+    if (ok && nj > 1) ok = load_k(1, &sh->k_full[1]);
+    static_assert(kVSlots == 2, "V slot j % 2 is also the parity of tile j");
     for (int j = 0; ok && j < nj; ++j) {
-      const int sv = j % kVSlots;
-      ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->v_empty[sv], ((j / kVSlots) & 1) ^ 1), 0);
+      const int b = j & 1;
+      ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->v_empty[b], ((j >> 1) & 1) ^ 1), 0);
       __syncwarp();
       if (!ok) break;
       if (leader) {
-        uint8_t* v = sV + sv * kTileBytes;
-        mbar_expect_tx(&sh->v_full[sv], kTileBytes);
-        tma_load_2d(v, &tmV, &sh->v_full[sv], x0, (j0 + j) * kAttnBN);
-        tma_load_2d(v + kTileBytes / 2, &tmV, &sh->v_full[sv], x0 + 64, (j0 + j) * kAttnBN);
+        uint8_t* v = sV + b * kTileBytes;
+        mbar_expect_tx(&sh->p_full[b][0], kTileBytes);
+        tma_load_2d(v, &tmV, &sh->p_full[b][0], x0, (j0 + j) * kAttnBN);
+        tma_load_2d(v + kTileBytes / 2, &tmV, &sh->p_full[b][0], x0 + 64, (j0 + j) * kAttnBN);
       }
-      if (j + 2 < nj) ok = load_k(j + 2);
+      if (j + 2 < nj) {
+        ok = load_k(j + 2, &sh->p_full[b][1]);
+      } else {
+        if (leader) mbar_arrive(&sh->p_full[b][1]);
+        __syncwarp();
+      }
     }
   } else if (warp == 1) {
     // MMA issuer: the whole warp runs the loop, waits and builds the descriptors (warp-uniform
@@ -241,9 +246,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       return r;
     };
+    // QK^T of tile j; tiles 0 and 1 wait for their K here, later ones through p_full
     auto issue_qk = [&](int j) -> bool {
       const int sk = j % kKSlots, b = j & 1;
-      if (!wait_all(&sh->k_full[sk], (j / kKSlots) & 1)) return false;
+      if (j < 2 && !wait_all(&sh->k_full[j], 0)) return false;
       tc_fence_after();
       const uint64_t kd = k_desc + (uint64_t)((sk * kTileBytes) >> 4);
       if (leader) {
@@ -270,8 +276,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool got = true;
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
+        // half 0 also brings V_j, half 1 also K_{j+2}
         if (!wait_all(&sh->p_full[b][q], (j >> 1) & 1)) { got = false; break; }
-        if (q == 0 && !wait_all(&sh->v_full[sv], (j / kVSlots) & 1)) { got = false; break; }
         tc_fence_after();
         if (leader) {
 #pragma unroll
