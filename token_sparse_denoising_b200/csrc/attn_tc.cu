@@ -7,8 +7,11 @@
 //   K, V: L x 128H cache rows, o: M x 128H.  Non-causal.
 //
 // One CTA = one head x 128 queries, streaming 128-key tiles of K and V.
-//   warp 0      TMA producer (the warp waits, one elected lane copies): Q once; K_j into a 3-slot ring, V_j into a 2-slot ring,
-//               in the order the MMA warp consumes them (K0 K1 V0 K2 V1 K3 ...)
+//   warp 0      TMA producer (the warp waits, one elected lane copies): Q once; K_j into a
+//               3-slot ring, V_j into a 2-slot ring, in the order the MMA warp consumes
+//               them (K0 K1 V0 K2 V1 K3 ...).  V_j and K_{j+2} complete on the barriers
+//               that also count the softmax warps' P stores of tile j, so the MMA warp
+//               waits twice per tile.
 //   warp 1      TMEM owner (512 columns) and MMA issuer (the warp runs the loop with
 //               warp-uniform descriptors, one elected lane issues):
 //                 S_b = Q K_j^T          (SS: both K-major, 128 x 128 x 128), b = j % 2
