@@ -169,7 +169,9 @@ def test_linear_f32(cuda_lib, M, K, Nout, epi):
 # ------------------------------------------------------------------ §2.2 attention
 
 @pytest.mark.parametrize("M,L,H,qscale", [(200, 1000, 2, 1.0), (128, 128, 1, 1.0), (1, 1, 1, 1.0),
-                                          (257, 300, 3, 4.0), (64, 4000, 2, 1.0)])
+                                          (257, 300, 3, 4.0), (64, 4000, 2, 1.0),
+                                          # two key tiles: each parity has one tile and no tile j+2
+                                          (130, 256, 2, 1.0), (100, 129, 1, 4.0)])
 def test_attention_bf16(cuda_lib, M, L, H, qscale):
     D = 128 * H
     q = S.normal(31, (M, D), qscale, True)
