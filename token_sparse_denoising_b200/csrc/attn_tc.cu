@@ -55,9 +55,10 @@ constexpr int kAttnThreads = 320;                 // 2 control warps + 8 softmax
 constexpr int kTileBytes = 128 * 128 * 2;         // one 128 x 128 bf16 operand tile (two 64-column boxes)
 constexpr uint32_t kColS = 0, kColO = 256;
 // Exponentials computed with the polynomial instead of the MUFU unit: the columns c
-// of a thread's 128 with (c % 8) >= 8 - kPolyPer8.  Measured at the Wan-1.3B shape
-// (attention alone, 32760 x 32760, 12 heads): 0 of 8 -> 6.44 ms, 2 of 8 -> 7.04 ms,
-// 4 of 8 -> 7.63 ms, so the MUFU path alone is the default.
+// of a thread's 128 with (c % 8) >= 8 - kPolyPer8.  Every measurement at the Wan-1.3B
+// shape (attention alone, 32760 x 32760, 12 heads) found the MUFU path faster: with two
+// softmax threads per row 0 / 2 / 4 of 8 took 6.44 / 7.04 / 7.63 ms, and with the tile
+// parities 6.05 / 6.35 / 7.52 ms at the power cap.  So the MUFU path alone is the default.
 #ifndef HSA_ATTN_POLY_PER8
 #define HSA_ATTN_POLY_PER8 0
 #endif
