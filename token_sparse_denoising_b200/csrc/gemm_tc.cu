@@ -7,9 +7,10 @@
 // Persistent CTAs (one per SM) walk 128 x BN output tiles.  Warp roles:
 //   warp 0      TMA producer: A (128 x 64) and B (BN x 64) k-blocks into a ring
 //               of STAGES shared-memory slots, 128-byte swizzled;
-//   warp 1      allocates 2 x BN TMEM columns (two accumulators); lane 0
-//               issues tcgen05.mma (M=128, N=BN, K=16) into the free one and
-//               releases each shared-memory slot with tcgen05.commit;
+//   warp 1      allocates 2 x BN TMEM columns (two accumulators); the warp runs
+//               the loop converged and one elected lane issues tcgen05.mma
+//               (M=128, N=BN, K=16) into the free one and releases each
+//               shared-memory slot with tcgen05.commit;
 //   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter, bias, GELU /
 //               residual gate.  Thread = output row.  Each warp stages 32 x 32
 //               sub-tiles of the output in shared memory and hands them to the TMA:
