@@ -53,6 +53,9 @@ def parse():
     p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the other workloads measured beside the headline (tiny loop, 30-block loop, "
+                        "Wan-14B block, attention and Euler sweeps)")
     p.add_argument("--mode", choices=["step", "loop", "sweep", "wan14", "tiny"], default="step",
                    help="step: the headline line; loop: 30-block Wan-1.3B loop, HSA vs uniform 40 steps; "
                         "sweep: attention + Euler kernel sweep; wan14: Wan-14B block active-fraction sweep; "
@@ -339,16 +342,19 @@ def run_gpu(args, rank, world, barrier, allmax):
     attn_per_step = attn_ms / args.steps
     achieved = attn_flops_per_full_step() / (attn_per_step * 1e-3) / 1e12
     traffic = traffic_per_launch()
+    timed_s = ms_step * args.steps / 1e3
     out = {
         "metric": METRIC, "value": round(ms_step, 4), "unit": "ms", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded random-init weights and inputs)",
         "config": workload_config(1.0),
         "roofline": {"bound": "tensor", "kernel": "k_attn_tc (self + cross attention launches)",
-                     "achieved": round(achieved, 1), "peak": peak_sus, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak_sus, 4),
-                     "peak_note": f"{src} sustained bf16 (burst {peak_burst}: frac {achieved / peak_burst:.3f}; "
-                                  f"datasheet dense bf16 2250: frac {achieved / 2250.0:.3f})",
+                     "achieved": round(achieved, 1), "peak": peak_burst, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_burst, 4),
+                     "peak_note": f"{src} burst bf16 (the timed region lasts {timed_s:.2f} s, too short for the "
+                                  f"sustained figure); of {src} sustained {peak_sus}: frac "
+                                  f"{achieved / peak_sus:.3f}; of datasheet dense bf16 2250: frac "
+                                  f"{achieved / 2250.0:.3f}",
                      "traffic": traffic, "launches_per_step": attn_n // max(args.steps, 1),
                      "flops_per_step": attn_flops_per_full_step()},
         "breakdown_ms_per_step": {"attention": round(attn_per_step, 4), "gemm": round(gemm_ms / args.steps, 4),
@@ -363,30 +369,44 @@ def run_gpu(args, rank, world, barrier, allmax):
     return out
 
 
-# ---------------------------------------------------------------- extra measurement modes
+# ---------------------------------------------------------------- the other workloads
 
-def run_loop(args):
+def _events():
+    import torch
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def measure_loop(graph: bool = True, n_blocks: int | None = None):
     """Full Wan-1.3B-shaped loop: latent 16x21x60x104 patchified 1x2x2 (N=32760, C=64), 30 blocks,
     T=40; HSA with budgets {40,20,10} sized 25/25/50 % and m=4 against the uniform 40-step run.
-    Each run is timed eagerly (host launches) and as one recorded CUDA graph of all T steps."""
+    Each run is timed eagerly (host launches) and, with `graph`, as one recorded CUDA graph of all
+    T steps.  Weights are drawn on the device (same recipe, N(0, 0.02^2))."""
     import torch
     from token_sparse_denoising_b200 import hsa, pipeline
     hsa.load()
     wl = S.WAN13_LOOP
     N = wl.grid.N
-    pm = S.patch_model_weights(wl.seed, wl.shape, wl.C, wl.n_blocks, True)
+    nb = wl.n_blocks if n_blocks is None else n_blocks
+    dev = torch.device("cuda", torch.cuda.current_device())
+    pm = S.patch_model_weights_on_device(wl.seed, wl.shape, wl.C, nb, True, dev)
     pos = S.token_positions(wl.grid)
-    ctx = S.normal(wl.seed * 10 + 3, (wl.shape.ctx_len, wl.shape.D), 1.0, True)
-    x0, vh0 = S.normal(wl.seed * 10 + 1, (N, wl.C)), S.normal(wl.seed * 10 + 2, (N, wl.C))
-    model = pipeline.PatchModel(pm, pos, N, bf16=True, ctx=ctx)
-    out = {"mode": "loop", "workload": f"{wl.name}: 30 blocks D=1536 H=12 F=8960 ctx=512, T=40, m=4, shift 5"}
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    ctx = S.device_normal(gen, (wl.shape.ctx_len, wl.shape.D), 1.0, True, dev)
+    x0 = S.device_normal(gen, (N, wl.C), 1.0, False, dev)
+    vh0 = S.device_normal(gen, (N, wl.C), 1.0, False, dev)
+    model = pipeline.PatchModel(pm, pos, N, bf16=True, ctx=ctx, device=dev)
+    del pm
+    out = {"workload": f"{wl.name}: {nb} blocks D=1536 H=12 F=8960 ctx=512, latent 16x21x60x104 patchified 1x2x2 "
+                       f"(N={N}, C=64), T=40, budgets {{40,20,10}} at 25/25/50 %, m=4, shifted sigma (shift 5)",
+           "weights": "device-drawn N(0, 0.02^2), seeded"}
     for name, budgets, fracs in (("hsa", wl.budgets, wl.fracs), ("uniform", (wl.T,), (1.0,))):
         sizes = S.group_sizes(N, fracs)
-        run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift)
+        run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift, device=dev)
         run.step()                                     # warm-up iteration (not timed)
-        run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift)
+        run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift, device=dev)
         torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a, b = _events()
         a.record()
         run.run()
         b.record()
@@ -394,34 +414,39 @@ def run_loop(args):
         assert hsa.device_status() == 0
         out[name] = {"ms": round(a.elapsed_time(b), 1), "token_steps": int(run.n_active.sum()),
                      "active_fraction": round(float(run.n_active.sum()) / (wl.T * N), 4)}
-        x_eager = run.x.clone()
-        # the same run recorded as one CUDA graph (every launch of all T steps) and replayed
-        run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift)
-        n0 = hsa.launch_count()
-        t0 = time.perf_counter()
-        g = run.capture()
-        torch.cuda.synchronize()
-        cap_s = time.perf_counter() - t0
-        recorded = hsa.launch_count() - n0
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        run.replay(g)
-        b.record()
-        b.synchronize()
-        assert hsa.device_status() == 0
-        out[name]["graph"] = {"ms": round(a.elapsed_time(b), 1), "capture_s": round(cap_s, 2),
-                              "launches_recorded": int(recorded),
-                              "bitwise_equal_to_eager": bool(torch.equal(run.x, x_eager))}
-        del g
+        if graph:
+            x_eager = run.x.clone()
+            run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift, device=dev)
+            n0 = hsa.launch_count()
+            t0 = time.perf_counter()
+            g = run.capture()
+            torch.cuda.synchronize()
+            cap_s = time.perf_counter() - t0
+            recorded = hsa.launch_count() - n0
+            a, b = _events()
+            a.record()
+            run.replay(g)
+            b.record()
+            b.synchronize()
+            assert hsa.device_status() == 0
+            out[name]["graph"] = {"ms": round(a.elapsed_time(b), 1), "capture_s": round(cap_s, 2),
+                                  "launches_recorded": int(recorded),
+                                  "bitwise_equal_to_eager": bool(torch.equal(run.x, x_eager))}
+            del g
     out["speedup"] = round(out["uniform"]["ms"] / out["hsa"]["ms"], 3)
-    out["speedup_graph"] = round(out["uniform"]["graph"]["ms"] / out["hsa"]["graph"]["ms"], 3)
+    out["ideal_speedup"] = round(out["uniform"]["token_steps"] / out["hsa"]["token_steps"], 3)
+    if graph:
+        out["speedup_graph"] = round(out["uniform"]["graph"]["ms"] / out["hsa"]["graph"]["ms"], 3)
+    del model
+    torch.cuda.empty_cache()
     return out
 
 
-def run_tiny(args):
-    """The tiny fp32 parity workload as a whole run: 4x16x16 tokens, D = 256, one block, T = 8, budgets
-    {8, 4} at 50/50 %, m = 1 (fp32 on the CUDA cores: a parity configuration, reported in ms only).
-    Timed eagerly and as one recorded CUDA graph, against the uniform 8-step run."""
+def measure_tiny(with_oracle: bool = True, reps: int = 5):
+    """The tiny fp32 workload as a whole run: 4x16x16 tokens, D = 256, one block, T = 8, budgets
+    {8, 4} at 50/50 %, m = 1 (fp32 on the CUDA cores).  Timed eagerly and as one recorded CUDA
+    graph, against the uniform 8-step run; with `with_oracle`, the oracle's whole loop on the host
+    cores beside it (the loop timed in full, no sampling)."""
     import torch
     from token_sparse_denoising_b200 import hsa, pipeline
     hsa.load()
@@ -431,16 +456,17 @@ def run_tiny(args):
     pos = S.token_positions(wl.grid)
     x0, vh0 = S.normal(wl.seed * 10 + 1, (N, D)), S.normal(wl.seed * 10 + 2, (N, D))
     model = pipeline.SingleBlockModel(bw, pos, N, bf16=False)
-    out = {"mode": "tiny", "workload": f"{wl.name}: N={N} (4x16x16) D={D} H=2 F=1024 fp32, T={wl.T}, m={wl.m}"}
+    out = {"workload": f"{wl.name}: N={N} (4x16x16) D={D} H=2 F=1024 fp32, T={wl.T}, budgets {{8,4}} at 50/50 %, "
+                       f"m={wl.m}, linear sigma"}
     for name, budgets, fracs in (("hsa", wl.budgets, wl.fracs), ("uniform", (wl.T,), (1.0,))):
         sizes = S.group_sizes(N, fracs)
         run = pipeline.HSARun(model, x0, vh0, wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift)
         run.run()                                      # warm-up run
         times = []
-        for _ in range(5):
+        for _ in range(reps):
             run.reset(x0, vh0)
             torch.cuda.synchronize()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a, b = _events()
             a.record()
             run.run()
             b.record()
@@ -449,10 +475,10 @@ def run_tiny(args):
         run.reset(x0, vh0)
         g = run.capture()
         gtimes = []
-        for _ in range(5):
+        for _ in range(reps):
             run.reset(x0, vh0)
             torch.cuda.synchronize()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a, b = _events()
             a.record()
             run.replay(g)
             b.record()
@@ -462,95 +488,144 @@ def run_tiny(args):
         assert hsa.device_status() == 0
         out[name] = {"ms": round(statistics.median(times), 3), "graph_ms": round(statistics.median(gtimes), 3),
                      "token_steps": int(run.n_active.sum())}
+        if with_oracle:
+            from oracle import hsa_oracle as O
+
+            def vel(xA, idx, caches):
+                o, Kc, Vc = O.dit_block_active(bw, xA, idx, pos, caches[0], caches[1])
+                return o, (Kc, Vc)
+
+            plan = O.make_plan(wl.T, budgets, sizes, wl.m, wl.sigma_kind, wl.shift, N)
+            z = np.zeros((N, D))
+            t0 = time.perf_counter()
+            O.hsa_denoise(x0, vh0, plan, vel, (z, z))
+            out[name]["oracle_ms"] = round((time.perf_counter() - t0) * 1e3, 1)
     out["speedup"] = round(out["uniform"]["ms"] / out["hsa"]["ms"], 3)
     out["speedup_graph"] = round(out["uniform"]["graph_ms"] / out["hsa"]["graph_ms"], 3)
+    if with_oracle:
+        out["oracle"] = {"kind": "oracle", "cores": blas_threads(), "sample": "the whole T = 8 loop, unsampled"}
     return out
 
 
-def run_sweep(args):
-    """Attention at N in {8190, 32760, 75600} x |A|/N in {1, .5, .25, .125} (12 heads, random active rows)
-    and the Euler update on N x 64 fp32 latents."""
+def measure_sweep(reps: int = 5):
+    """Attention at N in {8190, 32760, 75600} x |A|/N in {1, .5, .25, .125} (12 heads, bf16 Q/K/V
+    N(0,1)) and the Euler update on N x 64 fp32 latents with the L2 flushed before each launch."""
     import torch
     from token_sparse_denoising_b200 import hsa
     hsa.load()
-    peak_burst = load_peaks()[1]
-    hbm = load_peaks()[2]
-    res = {"mode": "sweep", "attention": [], "euler": []}
+    _, peak_burst, hbm, src = load_peaks()
+    res = {"attention": [], "euler": [], "peaks": f"{src}: burst bf16 {peak_burst} TFLOP/s, HBM {hbm} GB/s"}
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
     for N in (8190, 32760, 75600):
-        k = torch.randn((N, 1536), device="cuda").to(torch.bfloat16)
-        v = torch.randn((N, 1536), device="cuda").to(torch.bfloat16)
+        k = S.device_normal(gen, (N, 1536), 1.0, True, "cuda")
+        v = S.device_normal(gen, (N, 1536), 1.0, True, "cuda")
         for f in (1.0, 0.5, 0.25, 0.125):
             M = S.active_fraction_rows(N, f)
-            q = torch.randn((M, 1536), device="cuda").to(torch.bfloat16)
+            q = S.device_normal(gen, (M, 1536), 1.0, True, "cuda")
             o = torch.empty_like(q)
-            reps = 5
             need = hsa.attention_workspace_size(M, N, 12, hsa.HSA_BF16)
             ws = torch.empty(need, dtype=torch.uint8, device="cuda") if need else None
             for _ in range(2):
                 hsa.attention(q, k, v, 12, o, ws=ws)
             ms = time_device(lambda: hsa.attention(q, k, v, 12, o, ws=ws), reps, lambda: None) / reps
             tf = 4.0 * M * N * 128 * 12 / (ms * 1e-3) / 1e12
-            res["attention"].append({"N": N, "frac": f, "M": M, "split_ws_bytes": int(need), "ms": round(ms, 4),
-                                     "tflops": round(tf, 1),
-                                     "frac_of_burst_peak": round(tf / peak_burst, 3)})
-        x = torch.randn((N, 64), device="cuda")
-        vh = torch.randn((N, 64), device="cuda")
-        flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda")   # > L2: evict between reps
+            res["attention"].append({"N": N, "frac": f, "M": M, "ms": round(ms, 4), "tflops": round(tf, 1),
+                                     "frac_of_burst": round(tf / peak_burst, 3)})
+        del k, v
+    flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda")      # 256 MB > L2: evicts between launches
+    for N in (8190, 32760, 75600):
+        x = torch.randn((N, 64), device="cuda", generator=gen)
+        vh = torch.randn((N, 64), device="cuda", generator=gen)
         times = []
-        for _ in range(5):
+        for _ in range(max(reps, 5)):
             # the flush keeps the GPU busy while the host enqueues the timed launch, so the
-            # event interval holds the kernel alone (no host submission gap)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            # event interval holds the kernel alone
+            a, b = _events()
             flush.zero_()
             a.record()
             hsa.euler_update(x, vh, None, None, -0.025)
             b.record()
             b.synchronize()
             times.append(a.elapsed_time(b))
-        ms = min(times)
-        res["euler"].append({"N": N, "C": 64, "ms": round(ms, 5), "bytes": 12 * N * 64,
-                             "gbs": round(12 * N * 64 / (ms * 1e-3) / 1e9, 1),
-                             "frac_of_hbm": round(12 * N * 64 / (ms * 1e-3) / 1e9 / hbm, 3)})
+        ms = statistics.median(times)
+        gbs = 12 * N * 64 / (ms * 1e-3) / 1e9
+        res["euler"].append({"N": N, "C": 64, "us": round(ms * 1e3, 2), "bytes": 12 * N * 64, "gbs": round(gbs, 1),
+                             "frac_of_hbm": round(gbs / hbm, 3), "l2": "flushed before each launch"})
+    del flush
+    torch.cuda.empty_cache()
     return res
 
 
-def run_wan14(args):
-    """Wan-14B block (D=5120, 40 heads, FFN 13824, no context) at |A|/N in {1, .5, .25, .125},
-    contiguous and scattered active sets: layer-step ms."""
+def measure_wan14(patterns=("contiguous", "scattered"), reps: int = 3):
+    """Wan-14B block (D=5120, 40 heads, FFN 13824, no context) at |A|/N in {1, .5, .25, .125}:
+    layer-step ms for contiguous and/or scattered active sets.  Weights drawn on the device."""
     import torch
     from token_sparse_denoising_b200 import hsa
     hsa.load()
     grid, shape = S.WAN13_GRID, S.WAN14_BLOCK
     N, D = grid.N, shape.D
-    w = hsa.LayerWeights(S.block_weights(4, shape, True), "cuda", True)
-    kc = torch.randn((N, D), device="cuda").to(torch.bfloat16)
-    vc = torch.randn((N, D), device="cuda").to(torch.bfloat16)
-    x = torch.randn((N, D), device="cuda")
-    pos = torch.from_numpy(S.token_positions(grid)).cuda()
-    ws = torch.empty(hsa.layer_step_workspace_size(N, D, shape.F, hsa.HSA_BF16), dtype=torch.uint8, device="cuda")
-    xA = torch.empty((N, D), device="cuda")
-    res = {"mode": "wan14", "workload": "wan14b-block N=32760 D=5120 H=40 F=13824", "points": []}
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = hsa.LayerWeights(S.block_weights_on_device(4, shape, True, dev), dev, True)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(14)
+    kc = S.device_normal(gen, (N, D), 1.0, True, dev)
+    vc = S.device_normal(gen, (N, D), 1.0, True, dev)
+    x = S.device_normal(gen, (N, D), 1.0, False, dev)
+    pos = torch.from_numpy(S.token_positions(grid)).to(dev)
+    ws = torch.empty(hsa.layer_step_workspace_size(N, D, shape.F, hsa.HSA_BF16), dtype=torch.uint8, device=dev)
+    xA = torch.empty((N, D), device=dev)
+    peak_burst = load_peaks()[1]
+    res = {"workload": "wan14b-block N=32760 (21x30x52) D=5120 H=40 F=13824, no context", "points": []}
     for f in (1.0, 0.5, 0.25, 0.125):
         M = S.active_fraction_rows(N, f)
-        for pattern in ("contiguous", "scattered"):
-            idx = torch.from_numpy((S.contiguous_mask if pattern == "contiguous" else S.scattered_mask)(46, N, M)).cuda()
+        for pattern in patterns:
+            idx = torch.from_numpy((S.contiguous_mask if pattern == "contiguous" else S.scattered_mask)(46, N, M)).to(dev)
             fn = lambda: hsa.layer_step(w, kc, vc, xA[:M], idx, pos, ws, x_src=x)
             fn()
-            ms = time_device(fn, 3, lambda: None) / 3
+            ms = time_device(fn, reps, lambda: None) / reps
             flops = 4.0 * M * N * 128 * 40 + 2.0 * M * (3 * D * D + D * D + 2 * D * shape.F)
-            res["points"].append({"frac": f, "pattern": pattern, "M": M, "ms": round(ms, 3),
-                                  "tflops": round(flops / (ms * 1e-3) / 1e12, 1)})
+            tf = flops / (ms * 1e-3) / 1e12
+            res["points"].append({"frac": f, "pattern": pattern, "M": M, "ms": round(ms, 3), "tflops": round(tf, 1),
+                                  "frac_of_burst": round(tf / peak_burst, 3)})
     assert hsa.device_status() == 0
+    del w, kc, vc, x, ws, xA
+    torch.cuda.empty_cache()
     return res
+
+
+def run_loop(args):
+    return {"mode": "loop", **measure_loop(graph=True)}
+
+
+def run_tiny(args):
+    return {"mode": "tiny", **measure_tiny(with_oracle=True)}
+
+
+def run_sweep(args):
+    return {"mode": "sweep", **measure_sweep()}
+
+
+def run_wan14(args):
+    return {"mode": "wan14", **measure_wan14()}
+
+
+def measure_configs():
+    """The other workloads, measured beside the headline step on the same GPU in the same run."""
+    t0 = time.perf_counter()
+    out = {"attention_euler_sweep": measure_sweep(), "wan14_block": measure_wan14(patterns=("contiguous",)),
+           "tiny_fp32_loop": measure_tiny(with_oracle=True), "wan13_loop": measure_loop(graph=False)}
+    out["wall_s"] = round(time.perf_counter() - t0, 1)
+    return out
 
 
 # ---------------------------------------------------------------- the oracle on the host cores
 
-# (tokens whose q/k/v projections, Euler update and score run; query rows whose attention, O-projection,
-# cross-attention and FFN run) per sample: ~10 s of host work for the baseline beside the GPU numbers,
-# ~1 s per step for the reference arm, whose whole run must end within minutes.
-BASELINE_SAMPLE = (32760, 512)
-REFERENCE_SAMPLE = (4096, 32)
+# One sample of a full iteration, used by both the CPU baseline beside the GPU numbers and the
+# reference arm: the q/k/v projections, Euler update and score of SAMPLE[0] tokens, and attention
+# over all N cache rows + O-projection + cross-attention + FFN of SAMPLE[1] query rows.
+SAMPLE = (4096, 128)
+BASELINE_SECONDS = 10.0          # host work of the CPU baseline: repeats of the sample
 
 
 def blas_threads() -> int:
@@ -564,15 +639,15 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def oracle_step_sample(inp, sample):
-    """Time the oracle on a bounded sample of one full iteration; return the extrapolated ms per step.
+def oracle_step_sample(inp, sample=SAMPLE):
+    """Time the oracle on a bounded sample of one full iteration.
 
-    Every part of the step is linear in the rows it touches, so each is timed on
-    a spread sample and scaled. `sample` = (n_proj, n_rows): the q/k/v projections
-    (LN, GEMM, RMSNorm, RoPE) and the cached Euler update + L1 score of n_proj
-    tokens (x N/n_proj); attention over all N cache rows + O-projection +
-    cross-attention + FFN of n_rows query rows (x N/n_rows); the regrouping runs
-    on all N scores.
+    Every part of the step is linear in the rows it touches, so each is timed on a spread
+    sample and scaled: the q/k/v projections (LN, GEMM, RMSNorm, RoPE) and the cached Euler
+    update + L1 score of n_proj tokens (x N/n_proj); attention over all N cache rows +
+    O-projection + cross-attention + FFN of n_rows query rows (x N/n_rows); the regrouping
+    runs on all N scores.  Returns the extrapolated ms per step, the sample's wall seconds
+    and the measured per-unit times.
     """
     from oracle import hsa_oracle as O
     N = GRID.N
@@ -597,37 +672,60 @@ def oracle_step_sample(inp, sample):
     t4 = time.perf_counter()
     per_token = (t1 - t0) + (t3 - t2)
     est_ms = (per_token * N / len(proj) + (t2 - t1) * N / len(qrows) + (t4 - t3)) * 1e3
-    sample = (f"fp64 numpy oracle; q/k/v projections + Euler/score of {len(proj)} of {N} tokens "
-              f"({per_token:.2f} s, x{N / len(proj):.1f}), attention over all {N} cache rows + O/cross/FFN of "
-              f"{len(qrows)} query rows ({t2 - t1:.2f} s, x{N / len(qrows):.0f}), regrouping of {N} scores "
-              f"({t4 - t3:.2f} s)")
-    return est_ms, (t4 - t0), sample
+    units = {"token_ms": per_token * 1e3 / len(proj), "query_row_ms": (t2 - t1) * 1e3 / len(qrows),
+             "regroup_ms": (t4 - t3) * 1e3}
+    return est_ms, (t4 - t0), units
+
+
+def _sample_text(reps, units):
+    N = GRID.N
+    return (f"fp64 numpy oracle, {reps} repeat(s) of one sample of a full iteration: q/k/v projections + "
+            f"Euler/score of {SAMPLE[0]} of {N} tokens (measured {units['token_ms']:.4f} ms per token, x{N}), "
+            f"attention over all {N} cache rows + O/cross/FFN of {SAMPLE[1]} query rows (measured "
+            f"{units['query_row_ms']:.3f} ms per row, x{N}), regrouping of {N} scores "
+            f"({units['regroup_ms']:.1f} ms); value = the linear extrapolation to one full step")
 
 
 def cpu_baseline(inp):
-    est_ms, wall, sample = oracle_step_sample(inp, BASELINE_SAMPLE)
-    return {"value": round(est_ms, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
-            "sample": sample, "wall_s": round(wall, 2)}
+    vals, units, wall = [], [], 0.0
+    while wall < BASELINE_SECONDS or len(vals) < 2:
+        v, w, u = oracle_step_sample(inp)
+        vals.append(v)
+        units.append(u)
+        wall += w
+    med = lambda key: statistics.median(u[key] for u in units)
+    u = {k: med(k) for k in units[0]}
+    return {"value": round(statistics.median(vals), 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
+            "sample": _sample_text(len(vals), u), "measured_per_unit_ms": {k: round(x, 5) for k, x in u.items()},
+            "wall_s": round(wall, 2)}
 
 
 def run_reference(args):
+    """The reference arm: the oracle as it stands on the host cores, one sample of a full
+    iteration per step (the same sample as the CPU baseline of the GPU line); the value is the
+    median of the steps' extrapolated ms per full step."""
     inp = synthetic_inputs()
     for _ in range(args.warmup):
-        oracle_step_sample(inp, REFERENCE_SAMPLE)
-    vals, wall, sample = [], 0.0, ""
+        oracle_step_sample(inp)
+    vals, units, wall = [], [], 0.0
     for _ in range(args.steps):
-        v, w, sample = oracle_step_sample(inp, REFERENCE_SAMPLE)
+        v, w, u = oracle_step_sample(inp)
         vals.append(v)
+        units.append(u)
         wall += w
-    value = float(np.mean(vals))
+    value = float(statistics.median(vals))
+    u = {k: statistics.median(x[k] for x in units) for k in units[0]}
     return {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "ms", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value, 1), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(1.0),
             "cpu_baseline": {"value": round(value, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
-                             "sample": sample},
+                             "sample": _sample_text(args.steps, u),
+                             "measured_per_unit_ms": {k: round(x, 5) for k, x in u.items()}},
             "e2e": {"value": round(value, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-            "wall_s": round(wall, 1)}
+            "timing_note": "each step times one bounded sample and extrapolates it to a full step, so "
+                           "ms_per_step x steps is far longer than the run; sample_wall_s is what was spent",
+            "sample_wall_s": round(wall, 1)}
 
 
 # ---------------------------------------------------------------- main
@@ -688,6 +786,8 @@ def main():
             dist.barrier()
             dist.destroy_process_group()
     if rank == 0:
+        if world == 1 and not args.no_configs:
+            out["configs"] = measure_configs()
         if world == 1 and not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_baseline(synthetic_inputs())
         print(json.dumps(out), flush=True)

@@ -30,6 +30,12 @@
  *     index outside [0, N), a bounded wait that ran out) never trap: the
  *     kernel skips the access, records the fault in a device status word and
  *     finishes; hsa_device_status() reports it after the stream drains.
+ *     A wait that ran out also raises a per-device abort flag so that no other
+ *     kernel can hang: until hsa_device_status() has been called (which reads
+ *     and clears both), every later pipelined kernel on that device (attention,
+ *     GEMM) returns early and leaves its outputs incomplete.  A caller that can
+ *     meet a stall should therefore read the status after every step, not only
+ *     at the end of a run, to know which step first went wrong.
  *   - Matrices in [out][in] layout (row o holds the weights of output o),
  *     dtype HSA_BF16 (tensor-core path) or HSA_F32 (CUDA-core path).  Biases,
  *     norm gains, modulation vectors, latents and velocities are float32.
@@ -180,7 +186,8 @@ typedef struct hsa_layer_weights {
 /* Context keys/values of the cross-attention, once per run:
  *   K2 = RMSNorm(ctx W_k2^T + b_k2) * g_k2,  V2 = ctx W_v2^T + b_v2
  *   d_ctx: L x D in dtype; d_w_kv2: [2D][D] (k rows then v rows); d_b_kv2 [2D]; d_g_k2 [D];
- *   outputs d_k2, d_v2: L x D in dtype.  Workspace: hsa_context_kv_workspace_size(L, D). */
+ *   outputs d_k2, d_v2: L x D in dtype.  Workspace: hsa_context_kv_workspace_size(L, D) bytes,
+ *   the fp32 size (L x 2D x 4), which covers both dtypes; the bf16 path needs only half of it. */
 size_t hsa_context_kv_workspace_size(int L, int D);
 int hsa_context_kv(const void* d_ctx, int L, int D, int dtype, const void* d_w_kv2,
                    const float* d_b_kv2, const float* d_g_k2, void* d_k2, void* d_v2, void* d_ws,
@@ -194,10 +201,12 @@ int hsa_context_kv(const void* d_ctx, int L, int D, int dtype, const void* d_w_k
  * workspace it uses a scratch array built into the library: 8 MiB
  * (hsa_context_kv_noalloc_max_bytes()), held by every GPU that loads libhsa until
  * the process exits.  It allocates nothing.
- *   - Arguments as hsa_context_kv, without the workspace.  L x 2D x 4 bytes must not
- *     exceed the scratch size, else HSA_EINVAL (e.g. L = 512 fits up to D = 2048).
+ *   - Arguments as hsa_context_kv, without the workspace.  The L x 2D projection in
+ *     the call's dtype (4 bytes an element for HSA_F32, 2 for HSA_BF16) must fit the
+ *     scratch, else HSA_EINVAL: L = 512 fits up to D = 2048 in fp32, D = 4096 in bf16.
  *   - The first call on a device looks up the scratch's device address (once per
- *     device, with that device current); make that first call before any stream
+ *     device, with that device current, and again after the device's context has been
+ *     replaced, e.g. by cudaDeviceReset); make that first call before any stream
  *     capture.
  *   - Every call shares the one scratch array and leaves its contents behind; the
  *     projection writes each scratch element before reading it, so no clearing is
@@ -279,6 +288,48 @@ int hsa_patch_embed(const float* d_x, const int32_t* d_idx, int M, int N, int C,
 int hsa_velocity_head(const float* d_X, int M, int D, int C, int dtype, const float* d_head_mod,
                       const void* d_w_out, const float* d_b_out, float* d_vA, void* d_ws,
                       size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ head parallelism (one block over G GPUs)
+ * The pages run each denoising model on one device; these calls let one block's heads be split
+ * over G GPUs (each rank holding H/G heads of W_q, W_k, W_v, the KV cache of those heads for all
+ * N tokens, the matching columns of W_o and 1/G of the FFN) with the collectives between them
+ * issued by the caller (all-gather of the LayerNorm output, reduce of the partial projections,
+ * sum of the q/k squares).  Not in the pages: a way to run the §2.2 step when one block does not
+ * fit a GPU's time budget.  Every call is a plain kernel on local memory.
+ *
+ * LayerNorm rows: d_out[r] = LN(X[r]) * (1 + d_mul) + d_add (modulate != 0) or
+ * LN(X[r]) * d_mul + d_add (affine), eps 1e-6, over D channels (D % 128 == 0), output in dtype.
+ * With d_x_src (N x D float32) the rows are first gathered, X[r] = d_x_src[d_idx[r]], and
+ * written to d_X (M x D float32). */
+int hsa_layernorm_rows(float* d_X, const float* d_x_src, const int32_t* d_idx, int M, int N, int D,
+                       const float* d_mul, const float* d_add, int modulate, int dtype, void* d_out,
+                       void* stream);
+
+/* Partial RMS statistics: d_ss[r * ss_stride] = sum_c d_in[r * in_stride + c]^2 for c < D
+ * (float32 sums of dtype inputs; D % 4 == 0, in_stride % 4 == 0). */
+int hsa_row_sumsq(const void* d_in, int in_stride, int M, int D, int dtype, float* d_ss, int ss_stride,
+                  void* stream);
+
+/* q/k RMSNorm with sums of squares taken over all D_total channels of the row (d_ss[2r] for q,
+ * d_ss[2r+1] for k: the ranks' partial sums added), times the local gains d_g_q, d_g_k [Dl];
+ * then 3D RoPE of each local 128-channel head at d_pos[d_idx[r]]; d_Q[r] = q (M x Dl),
+ * d_kcache[d_idx[r]] = k, d_vcache[d_idx[r]] = v (N x Dl).  d_qkv rows are [q | k | v], Dl each
+ * (Dl % 128 == 0).  Rows of skipped tokens are not touched; indices outside [0, N) are flagged
+ * (HSA_EINDEX) and skipped. */
+int hsa_qk_norm_rope_ext(const void* d_qkv, int M, int N, int Dl, int D_total, const float* d_ss,
+                         const float* d_g_q, const float* d_g_k, const int32_t* d_idx,
+                         const int32_t* d_pos, int dtype, void* d_Q, void* d_kcache, void* d_vcache,
+                         void* stream);
+
+/* d_out[r] (M x D, dense) = d_in[r] * rsqrt(d_ss[r * ss_stride] / D_total + 1e-6) * d_g
+ * (d_g NULL = 1); with d_ss NULL a plain copy of the D first elements of each input row. */
+int hsa_rms_rows_ext(const void* d_in, int in_stride, int M, int D, int D_total, const float* d_ss,
+                     int ss_stride, const float* d_g, int dtype, void* d_out, void* stream);
+
+/* Residual update of reduced partial projections: d_X[r] += d_gate * (d_y[r] + d_b) over D
+ * channels (M x D float32 both; d_b, d_gate NULL = 0, 1). */
+int hsa_gated_residual(float* d_X, const float* d_y, int M, int D, const float* d_b,
+                       const float* d_gate, void* stream);
 
 #ifdef __cplusplus
 }

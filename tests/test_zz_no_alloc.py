@@ -43,8 +43,9 @@ def _without_workspace(ctx, w):
 
 
 def test_no_alloc_context_kv_matches_workspace_version(cuda_lib):
-    # two calls in a row with different inputs and sizes: the second reuses the scratch
-    for seed, L, D in ((3, 512, 1536), (9, 77, 256)):
+    # calls in a row with different inputs and sizes: each later call reuses the scratch; the
+    # last one fills it exactly (bf16: 512 x 2 x 4096 x 2 bytes = 8 MiB)
+    for seed, L, D in ((3, 512, 1536), (9, 77, 256), (11, 512, 4096)):
         ctx, w = _case(seed, L, D)
         k_ref, v_ref = _with_workspace(ctx, w)
         k, v = _without_workspace(ctx, w)
@@ -55,8 +56,8 @@ def test_no_alloc_context_kv_matches_workspace_version(cuda_lib):
 
 def test_no_alloc_rejects_oversize(cuda_lib):
     assert hsa.lib().hsa_context_kv_noalloc_max_bytes() == 8 << 20
-    ctx, w = _case(5, 8192, 256)            # 8192 x 512 x 4 bytes = 16 MiB > 8 MiB
-    k = torch.empty((8192, 256), dtype=torch.bfloat16, device="cuda")
+    ctx, w = _case(5, 8192, 512)            # bf16: 8192 x 1024 x 2 bytes = 16 MiB > 8 MiB
+    k = torch.empty((8192, 512), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(hsa.HsaError) as e:
         hsa.context_kv_noalloc(ctx, w.t["w_kv2"], w.t["b_kv2"], w.t["g_k2"], k, torch.empty_like(k))
     assert e.value.code == hsa.HSA_EINVAL

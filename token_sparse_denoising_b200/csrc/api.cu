@@ -164,6 +164,15 @@ extern "C" size_t hsa_context_kv_workspace_size(int L, int D) {
   return align256((size_t)L * 2 * D * 4);
 }
 
+namespace hsa {
+// Scratch the context projection really uses: the L x 2D projection in the path's own dtype.
+// hsa_context_kv_workspace_size reports the fp32 size, which covers both dtypes.
+size_t context_kv_scratch_bytes(int L, int D, int dtype) {
+  if (L <= 0 || D <= 0) return 0;
+  return align256((size_t)L * 2 * D * esize(dtype));
+}
+}  // namespace hsa
+
 extern "C" int hsa_context_kv(const void* d_ctx, int L, int D, int dtype, const void* d_w_kv2, const float* d_b_kv2,
                               const float* d_g_k2, void* d_k2, void* d_v2, void* d_ws, size_t ws_bytes,
                               void* stream) {
@@ -171,7 +180,7 @@ extern "C" int hsa_context_kv(const void* d_ctx, int L, int D, int dtype, const 
   if (L <= 0 || D <= 0 || D % 128) return set_error(HSA_EINVAL, "context_kv: need L > 0 and D % 128 == 0");
   if (!d_ctx || !d_w_kv2 || !d_g_k2 || !d_k2 || !d_v2 || !d_ws)
     return set_error(HSA_EINVAL, "context_kv: null pointer");
-  if (ws_bytes < hsa_context_kv_workspace_size(L, D)) return set_error(HSA_EWORKSPACE, "context_kv: workspace");
+  if (ws_bytes < context_kv_scratch_bytes(L, D, dtype)) return set_error(HSA_EWORKSPACE, "context_kv: workspace");
   cudaStream_t st = as_stream(stream);
   HSA_TRY(linear(d_ctx, L, D, d_w_kv2, 2 * D, d_b_kv2, dtype, HSA_EPI_STORE, nullptr, d_ws, st));
   if (dtype == HSA_BF16) {

@@ -556,15 +556,13 @@ int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, in
   if (!rc) rc = make_tmap_2d(&tk, K, true, D, (uint64_t)L, D * 2, 64, kAttnBN, true);
   if (!rc) rc = make_tmap_2d(&tv, V, true, D, (uint64_t)L, D * 2, 64, kAttnBN, true);
   if (rc) return rc;
-  static bool attr_done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return set_error(HSA_ECUDA, "attention: device index out of range");
-  if (!attr_done[dev]) {
+  static PerContextOnce attr;
+  rc = attr.ensure([](void**) {
     if (cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess)
       return check_launch("attention: shared-memory attribute");
-    attr_done[dev] = true;
-  }
+    return (int)HSA_OK;
+  });
+  if (rc) return rc;
   const int QT = (M + kAttnBM - 1) / kAttnBM, U = QT * H;
   TailSplit ts = plan_tail(U, (L + kAttnBN - 1) / kAttnBN, num_sms());
   const size_t need = tail_split_bytes(ts);

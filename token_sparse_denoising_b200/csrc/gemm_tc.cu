@@ -241,14 +241,13 @@ template <int BN, int EPI>
 static int launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, int M, int Nout,
                           int K, const float* bias, const float* gate, void* out, cudaStream_t st) {
   auto kern = k_gemm_tc<BN, EPI>;
-  static bool attr_done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+  static PerContextOnce attr;
+  const int arc = attr.ensure([&](void**) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<BN>::kSmem) != cudaSuccess)
       return check_launch("gemm: shared-memory attribute");
-    attr_done[dev] = true;
-  }
+    return (int)HSA_OK;
+  });
+  if (arc) return arc;
   const int tiles = (Nout / BN) * ((M + kGemmBM - 1) / kGemmBM);
   dim3 grid(tiles < num_sms() ? tiles : num_sms());
   ScopedTiming timing(HSA_KCLASS_GEMM, st);

@@ -8,4 +8,5 @@
 #include "attn_tc.cu"
 #include "simt_f32.cu"
 #include "api.cu"
+#include "shard.cu"
 #include "noalloc.cu"

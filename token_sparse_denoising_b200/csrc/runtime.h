@@ -5,7 +5,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <string>
+
+#include "../../include/hsa.h"
 
 namespace hsa {
 
@@ -13,6 +16,43 @@ int set_error(int code, const std::string& msg);
 int check_launch(const char* what);
 void count_launch(int n);
 int num_sms();
+
+// Identity of the current CUDA context, unique for the life of the process (cuCtxGetId): a
+// device reset or a new primary context gives a new value.  0 when no context is current yet
+// or the driver cannot say.
+uint64_t current_context_id();
+
+// Host set-up that must run once per CUDA context of a device -- a kernel attribute, the
+// device address of a __device__ symbol -- shared by every host thread.  ensure(setup, &v)
+// calls setup(&v) under a lock when the current device's context is not the one the last
+// successful set-up ran in (after cudaDeviceReset, for instance), or when the context's
+// identity cannot be read; otherwise it returns the value that set-up stored.
+class PerContextOnce {
+ public:
+  template <typename F>
+  int ensure(F&& setup, void** out = nullptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+      return set_error(HSA_ECUDA, "no usable current CUDA device");
+    const uint64_t id = current_context_id();
+    std::lock_guard<std::mutex> g(mu_);
+    if (id == 0 || ctx_[dev] != id) {
+      void* v = nullptr;
+      const int rc = setup(&v);
+      if (rc != HSA_OK) return rc;
+      ctx_[dev] = id;
+      value_[dev] = v;
+    }
+    if (out) *out = value_[dev];
+    return HSA_OK;
+  }
+
+ private:
+  static constexpr int kMaxDevices = 64;
+  std::mutex mu_;
+  uint64_t ctx_[kMaxDevices] = {};
+  void* value_[kMaxDevices] = {};
+};
 
 // 2-D tiled tensor map over a row-major matrix of `outer` rows x `inner` elements
 // (bf16 or f32), rows `row_stride_bytes` apart, boxes of box_outer x box_inner.

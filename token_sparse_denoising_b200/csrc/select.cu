@@ -400,15 +400,14 @@ extern "C" int hsa_select_tokens_pinned(const float* d_score, const uint8_t* d_p
   a.staged = N <= kSelectStagedMax ? 1 : 0;
   constexpr size_t kHistBytes = (size_t)(kSelectThreads / 32) * kHistStride * sizeof(uint32_t);
   const size_t dyn = kHistBytes + (a.staged ? (size_t)N * sizeof(uint32_t) : 0);
-  static bool attr_done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+  static PerContextOnce attr;
+  const int arc = attr.ensure([](void**) {
     if (cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kHistBytes + kSelectStagedMax * (int)sizeof(uint32_t)) != cudaSuccess)
       return check_launch("select: shared-memory attribute");
-    attr_done[dev] = true;
-  }
+    return (int)HSA_OK;
+  });
+  if (arc) return arc;
   ScopedTiming timing(HSA_KCLASS_OTHER, as_stream(stream));
   k_select<<<1, kSelectThreads, dyn, as_stream(stream)>>>(d_score, d_pinned, N, a, d_group, d_order);
   count_launch(1);

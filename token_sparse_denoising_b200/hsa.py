@@ -64,6 +64,11 @@ _SIGS = {
     "hsa_patch_workspace_size": (sz, [i32, i32, i32, i32]),
     "hsa_patch_embed": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]),
     "hsa_velocity_head": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
+    "hsa_layernorm_rows": (i32, [vp, vp, vp, i32, i32, i32, vp, vp, i32, i32, vp, vp]),
+    "hsa_row_sumsq": (i32, [vp, i32, i32, i32, i32, vp, i32, vp]),
+    "hsa_qk_norm_rope_ext": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]),
+    "hsa_rms_rows_ext": (i32, [vp, i32, i32, i32, i32, vp, i32, vp, i32, vp, vp]),
+    "hsa_gated_residual": (i32, [vp, vp, i32, i32, vp, vp, vp]),
 }
 
 
@@ -295,6 +300,52 @@ def velocity_head(X, head_mod, w_out, b_out, vA, ws, stream=None):
                                    _stream(stream)), "hsa_velocity_head")
 
 
+def _device_copy(a, device, dtype):
+    """A contiguous device tensor of `dtype` from a numpy array or a torch tensor."""
+    import torch
+    if isinstance(a, torch.Tensor):
+        return a.to(device=device, dtype=dtype).contiguous()
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device).to(dtype)
+
+
+# ---------------------------------------------------------------- head-parallel building blocks
+
+def layernorm_rows(X, mul, add, out, modulate: bool, x_src=None, idx=None, stream=None):
+    """out = LN(X)(1 + mul) + add (modulate) or LN(X) mul + add; with x_src, X = x_src[idx] first."""
+    M, D = X.shape
+    N = 0 if x_src is None else x_src.shape[0]
+    _check(lib().hsa_layernorm_rows(_ptr(X), _ptr(x_src), _ptr(idx), M, N, D, _ptr(mul), _ptr(add),
+                                    1 if modulate else 0, _dtype_code(out), _ptr(out), _stream(stream)),
+           "hsa_layernorm_rows")
+
+
+def row_sumsq(x, D: int, ss, ss_stride: int = 1, stream=None):
+    """ss[r * ss_stride] = sum of squares of the first D elements of row r of x (2-D, any width)."""
+    M = x.shape[0]
+    _check(lib().hsa_row_sumsq(_ptr(x), x.stride(0), M, D, _dtype_code(x), _ptr(ss), ss_stride, _stream(stream)),
+           "hsa_row_sumsq")
+
+
+def qk_norm_rope_ext(qkv, M: int, D_total: int, ss, g_q, g_k, idx, pos, Q, kcache, vcache, stream=None):
+    Dl = qkv.shape[1] // 3
+    N = kcache.shape[0]
+    _check(lib().hsa_qk_norm_rope_ext(_ptr(qkv), M, N, Dl, D_total, _ptr(ss), _ptr(g_q), _ptr(g_k), _ptr(idx),
+                                      _ptr(pos), _dtype_code(qkv), _ptr(Q), _ptr(kcache), _ptr(vcache),
+                                      _stream(stream)), "hsa_qk_norm_rope_ext")
+
+
+def rms_rows_ext(x, M: int, D: int, D_total: int, ss, g, out, ss_stride: int = 1, stream=None):
+    """out[:M] = x[:M, :D] * rsqrt(ss / D_total + eps) * g (ss None: a plain copy)."""
+    _check(lib().hsa_rms_rows_ext(_ptr(x), x.stride(0), M, D, D_total, _ptr(ss), ss_stride, _ptr(g),
+                                  _dtype_code(x), _ptr(out), _stream(stream)), "hsa_rms_rows_ext")
+
+
+def gated_residual(X, y, b=None, gate=None, stream=None):
+    M, D = X.shape
+    _check(lib().hsa_gated_residual(_ptr(X), _ptr(y), M, D, _ptr(b), _ptr(gate), _stream(stream)),
+           "hsa_gated_residual")
+
+
 class LayerWeights:
     """Device copies of one block's parameters plus the C struct that points at them."""
 
@@ -308,16 +359,15 @@ class LayerWeights:
         for name in self.MATS:
             a = getattr(bw, name)
             if a is not None:
-                self.t[name] = torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device).to(mat_dtype)
+                self.t[name] = _device_copy(a, device, mat_dtype)
         for name in self.VECS:
             a = getattr(bw, name)
             if a is not None:
-                self.t[name] = torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
-        for name in ("w_kv2",):
-            if getattr(bw, name) is not None:
-                self.t[name] = torch.from_numpy(np.ascontiguousarray(bw.w_kv2, np.float32)).to(device).to(mat_dtype)
-                self.t["b_kv2"] = torch.from_numpy(np.ascontiguousarray(bw.b_kv2, np.float32)).to(device)
-                self.t["g_k2"] = torch.from_numpy(np.ascontiguousarray(bw.g_k2, np.float32)).to(device)
+                self.t[name] = _device_copy(a, device, torch.float32)
+        if bw.w_kv2 is not None:
+            self.t["w_kv2"] = _device_copy(bw.w_kv2, device, mat_dtype)
+            self.t["b_kv2"] = _device_copy(bw.b_kv2, device, torch.float32)
+            self.t["g_k2"] = _device_copy(bw.g_k2, device, torch.float32)
         D, F = bw.w_o.shape[0], bw.w_1.shape[0]
         self.D, self.H, self.F = D, D // 128, F
         self.dtype = HSA_BF16 if bf16 else HSA_F32

@@ -22,6 +22,8 @@ from . import hsa
 
 
 def _to_dev(a, dtype=torch.float32, device="cuda"):
+    if isinstance(a, torch.Tensor):
+        return a.to(device=device, dtype=dtype).contiguous()
     return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device).to(dtype)
 
 
@@ -186,6 +188,8 @@ class HSARun:
         i = self.i
         idx = self.active_index(i)
         full = idx.shape[0] == self.N
+        # a prefix view of `order`, which the regrouping below rewrites: copy it out first
+        idx_rec = idx.cpu().numpy().copy() if record is not None else None
         vA = self.model.velocity(self.x, idx)
         dsig = float(np.float32(self.sigmas[i + 1]) - np.float32(self.sigmas[i]))
         regroup = full and self.static_order is None
@@ -193,7 +197,7 @@ class HSARun:
         if regroup:
             hsa.select_tokens(self.score, self.sizes, self.group, self.order, ws=self.sel_ws, pinned=self.pinned)
         if record is not None:
-            record.append({"i": i, "M": int(idx.shape[0]), "full": full,
+            record.append({"i": i, "M": int(idx.shape[0]), "full": full, "idx": idx_rec,
                            "score": self.score.cpu().numpy().copy() if regroup else None,
                            "order": self.order.cpu().numpy().copy()})
         self.i += 1

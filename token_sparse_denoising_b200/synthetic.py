@@ -29,11 +29,15 @@ ROPE_SPLIT = (44, 42, 42)
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round float32 values to bf16 (nearest, ties to even); returns uint16 bit patterns."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    nan = np.isnan(a)
-    out = rounded.astype(np.uint16)
-    out[nan] = 0x7FC0
+    u = a.view(np.uint32)
+    # u + 0x7FFF + lsb stays below 2^32 for every non-NaN pattern (the largest, -inf, is
+    # 0xFF800000), so 32-bit arithmetic is exact; NaNs are replaced afterwards
+    t = (u >> 16) & np.uint32(1)
+    t += np.uint32(0x7FFF)
+    t += u
+    t >>= 16
+    out = t.astype(np.uint16)
+    out[np.isnan(a)] = 0x7FC0
     return out
 
 
@@ -181,6 +185,55 @@ def patch_model_weights(seed: int, shape: BlockShape, C: int, n_blocks: int, bf1
         head_mod=normal(s + 1, (2, shape.D), std, False),
         w_out=normal(s + 2, (C, shape.D), std, bf16), b_out=np.zeros(C, np.float32),
         blocks=[block_weights(s + 8 + b, shape, bf16, std) for b in range(n_blocks)])
+
+
+# ---------------------------------------------------------------- draws on the device
+
+def device_normal(gen, shape, scale: float, bf16: bool, device):
+    """N(0, scale^2) drawn on the device by torch's seeded generator `gen`; bf16 (rounded to
+    nearest even) or float32."""
+    import torch
+    t = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+    t.mul_(scale)
+    return t.to(torch.bfloat16) if bf16 else t
+
+
+def block_weights_on_device(seed: int, shape: BlockShape, bf16: bool, device, std: float = 0.02) -> BlockWeights:
+    """The recipe of block_weights drawn on the device (torch tensors; other values than the
+    numpy draws of the same seed).  For measurements, where only shapes and distributions
+    matter and drawing hundreds of millions of values on the host would take minutes."""
+    import torch
+    D, F = shape.D, shape.F
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1_000_003 * (seed + 1))
+    z = lambda n: torch.zeros(n, dtype=torch.float32, device=device)
+    one = lambda n: torch.ones(n, dtype=torch.float32, device=device)
+    nrm = lambda shp, b: device_normal(gen, shp, std, b, device)
+    bw = BlockWeights(
+        w_qkv=nrm((3 * D, D), bf16), b_qkv=z(3 * D), g_q=one(D), g_k=one(D),
+        w_o=nrm((D, D), bf16), b_o=z(D), w_1=nrm((F, D), bf16), b_1=z(F),
+        w_2=nrm((D, F), bf16), b_2=z(D), mod=nrm((6, D), False), shape=shape)
+    if shape.cross:
+        bw.ln_c_g, bw.ln_c_b = one(D), z(D)
+        bw.w_q2, bw.b_q2, bw.g_q2 = nrm((D, D), bf16), z(D), one(D)
+        bw.w_kv2, bw.b_kv2, bw.g_k2 = nrm((2 * D, D), bf16), z(2 * D), one(D)
+        bw.w_o2, bw.b_o2 = nrm((D, D), bf16), z(D)
+    return bw
+
+
+def patch_model_weights_on_device(seed: int, shape: BlockShape, C: int, n_blocks: int, bf16: bool, device,
+                                  std: float = 0.02) -> PatchModelWeights:
+    """patch_model_weights drawn on the device (see block_weights_on_device)."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(2_000_003 * (seed + 1))
+    return PatchModelWeights(
+        w_in=device_normal(gen, (shape.D, C), std, bf16, device),
+        b_in=torch.zeros(shape.D, dtype=torch.float32, device=device),
+        head_mod=device_normal(gen, (2, shape.D), std, False, device),
+        w_out=device_normal(gen, (C, shape.D), std, bf16, device),
+        b_out=torch.zeros(C, dtype=torch.float32, device=device),
+        blocks=[block_weights_on_device(100 * seed + 8 + b, shape, bf16, device, std) for b in range(n_blocks)])
 
 
 # ---------------------------------------------------------------- named workloads
