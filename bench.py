@@ -533,7 +533,21 @@ def measure_sweep(reps: int = 5):
             res["attention"].append({"N": N, "frac": f, "M": M, "ms": round(ms, 4), "tflops": round(tf, 1),
                                      "frac_of_burst": round(tf / peak_burst, 3)})
         del k, v
+    # the cross-attention shape: every active query against the 512-row text context
+    M, L = S.WAN13_GRID.N, S.WAN13_BLOCK.ctx_len
+    k = S.device_normal(gen, (L, 1536), 1.0, True, "cuda")
+    v = S.device_normal(gen, (L, 1536), 1.0, True, "cuda")
+    q = S.device_normal(gen, (M, 1536), 1.0, True, "cuda")
+    o = torch.empty_like(q)
+    for _ in range(2):
+        hsa.attention(q, k, v, 12, o)
+    ms = time_device(lambda: hsa.attention(q, k, v, 12, o), 4 * reps, lambda: None) / (4 * reps)
+    tf = 4.0 * M * L * 128 * 12 / (ms * 1e-3) / 1e12
+    res["cross_attention"] = {"M": M, "L": L, "H": 12, "ms": round(ms, 4), "tflops": round(tf, 1),
+                              "frac_of_burst": round(tf / peak_burst, 3)}
+    del q, k, v, o
     flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda")      # 256 MB > L2: evicts between launches
+    flush_r = torch.zeros(256 * 1024 * 1024 // 4, device="cuda")
     for N in (8190, 32760, 75600):
         x = torch.randn((N, 64), device="cuda", generator=gen)
         vh = torch.randn((N, 64), device="cuda", generator=gen)
@@ -543,6 +557,7 @@ def measure_sweep(reps: int = 5):
             # event interval holds the kernel alone
             a, b = _events()
             flush.zero_()
+            flush_r.sum()              # read over the dirty lines: they are written back here, not in the launch
             a.record()
             hsa.euler_update(x, vh, None, None, -0.025)
             b.record()
@@ -550,9 +565,35 @@ def measure_sweep(reps: int = 5):
             times.append(a.elapsed_time(b))
         ms = statistics.median(times)
         gbs = 12 * N * 64 / (ms * 1e-3) / 1e9
-        res["euler"].append({"N": N, "C": 64, "us": round(ms * 1e3, 2), "bytes": 12 * N * 64, "gbs": round(gbs, 1),
-                             "frac_of_hbm": round(gbs / hbm, 3), "l2": "flushed before each launch"})
-    del flush
+        entry = {"N": N, "C": 64, "us": round(ms * 1e3, 2), "bytes": 12 * N * 64, "gbs": round(gbs, 1),
+                 "frac_of_hbm": round(gbs / hbm, 3),
+                 "l2": "written (256 MB) then read (256 MB) before each launch, so no dirty line of the flush is "
+                       "written back inside the timed launch"}
+        del x, vh
+        # back to back, as in a run: launches over distinct (x, v_hat) sets whose total is >= 2x L2
+        sets = max(2, (512 << 20) // (8 * N * 64))
+        xs = [torch.randn((N, 64), device="cuda", generator=gen) for _ in range(sets)]
+        vs = [torch.randn((N, 64), device="cuda", generator=gen) for _ in range(sets)]
+        for _ in range(2):
+            for k in range(sets):
+                hsa.euler_update(xs[k], vs[k], None, None, -0.025)
+        bt = []
+        for _ in range(5):
+            a, b = _events()
+            a.record()
+            for k in range(sets):
+                hsa.euler_update(xs[k], vs[k], None, None, -0.025)
+            b.record()
+            b.synchronize()
+            bt.append(a.elapsed_time(b) / sets)
+        ms_b = statistics.median(bt)
+        gbs_b = 12 * N * 64 / (ms_b * 1e-3) / 1e9
+        entry["back_to_back"] = {"us_per_launch": round(ms_b * 1e3, 2), "gbs": round(gbs_b, 1),
+                                 "frac_of_hbm": round(gbs_b / hbm, 3), "sets": sets,
+                                 "working_set_mb": round(sets * 8 * N * 64 / 1e6, 1)}
+        res["euler"].append(entry)
+        del xs, vs
+    del flush, flush_r
     torch.cuda.empty_cache()
     return res
 
