@@ -205,12 +205,12 @@ def test_attention_identical_keys_give_mean_value(cuda_lib):
     assert max_abs(host(o), np.tile(v.astype(np.float64).mean(0), (M, 1))) < 1e-2
 
 
-@pytest.mark.parametrize("M,L,H", [(1000, 4000, 12), (300, 1000, 2), (300, 512, 2), (129, 2000, 3)])
+@pytest.mark.parametrize("M,L,H", [(1000, 4000, 12), (300, 1100, 2), (100, 1536, 2), (129, 2000, 3)])
 def test_attention_split_tail_matches_oracle(cuda_lib, M, L, H):
     """With a workspace the units of the last, incomplete wave are split over key ranges and
-    merged by a second kernel (1000 x 4000 x 12 heads: 96 units, 3 ranges each; 300 x 1000: the
-    last range holds the ragged key tile; 300 x 512: ranges of two tiles).  Checked against the
-    oracle, and against the unsplit kernel to fp32-merge rounding."""
+    merged by a second kernel (1000 x 4000 x 12 heads: 96 units, 3 ranges each; 300 x 1100: the
+    last range holds the ragged key tile; 100 x 1536: one query tile, ranges of two tiles).
+    Checked against the oracle, and against the unsplit kernel to fp32-merge rounding."""
     D = 128 * H
     q = S.normal(71, (M, D), 1.0, True)
     k, v = S.normal(72, (L, D), 1.0, True), S.normal(73, (L, D), 1.0, True)
@@ -232,6 +232,37 @@ def test_attention_split_tail_matches_oracle(cuda_lib, M, L, H):
     assert torch.equal(o2, o1)
 
 
+@pytest.mark.parametrize("M,L,H", [(256, 512, 12), (300, 16, 2), (200, 300, 2), (2000, 1000, 3), (129, 1024, 1),
+                                   (640, 129, 2)])
+def test_attention_two_query_tiles(cuda_lib, M, L, H):
+    """Key ranges of at most 8 tiles (the cross-attention's context) run two query tiles per CTA,
+    each key tile loaded once for both: exact multiples of 256 queries, a ragged second query
+    tile (300, 200, 2000 rows; 129 rows: a pair with a single real row), a single ragged key tile
+    (16 keys), the largest range that takes this path (1024 keys) and a ragged 129-key range."""
+    D = 128 * H
+    q = S.normal(91, (M, D), 2.0, True)
+    k, v = S.normal(92, (L, D), 1.0, True), S.normal(93, (L, D), 1.0, True)
+    assert cuda_lib.attention_workspace_size(M, L, H, cuda_lib.HSA_BF16) == 0      # no key-range split
+    o = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    cuda_lib.attention(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), H, o)
+    assert cuda_lib.device_status() == 0
+    assert_bf16_close(host(o), O.attention(q, k, v), "attention, two query tiles per CTA")
+
+
+def test_attention_two_query_tiles_wan_cross(cuda_lib):
+    """The Wan-1.3B cross-attention shape: 32760 queries against the 512-row context, 12 heads
+    (64 pairs of query tiles per head, the last one ragged); sampled rows against the oracle."""
+    M, L, H = 32760, 512, 12
+    D = 128 * H
+    q = S.normal(94, (M, D), 1.0, True)
+    k, v = S.normal(95, (L, D), 1.0, True), S.normal(96, (L, D), 1.0, True)
+    o = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    cuda_lib.attention(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), H, o)
+    assert cuda_lib.device_status() == 0
+    rows = np.array([0, 127, 128, 255, 256, 16000, 32639, 32640, 32700, 32759])
+    assert_bf16_close(host(o)[rows], O.attention(q[rows], k, v), "cross-attention shape, sampled rows")
+
+
 def test_attention_split_tail_wan_quarter(cuda_lib):
     """The Wan-1.3B shape at |A|/N = 1/4 (8190 queries, 32760 keys, 12 heads): 768 units, the 28
     of the incomplete last wave split 5 ways; sampled rows against the oracle."""
@@ -251,10 +282,26 @@ def test_attention_split_tail_wan_quarter(cuda_lib):
     assert_bf16_close(got, want, "split attention, sampled rows")
 
 
-@pytest.mark.parametrize("M,L,H", [(100, 300, 2), (1, 1024, 1)])
+@pytest.mark.parametrize("M,L,H", [(100, 300, 2), (1, 1024, 1), (33, 65, 1)])
 def test_attention_f32(cuda_lib, M, L, H):
     D = 128 * H
     q, k, v = S.normal(61, (M, D)), S.normal(62, (L, D)), S.normal(63, (L, D))
     o = torch.empty((M, D), device="cuda")
     cuda_lib.attention(dev(q), dev(k), dev(v), H, o)
+    assert_f32_close(host(o), O.attention(q, k, v))
+
+
+@pytest.mark.parametrize("M,L,H", [(1024, 1024, 2), (512, 1024, 2), (37, 300, 3), (1, 200, 1)])
+def test_attention_f32_key_range_split(cuda_lib, M, L, H):
+    """fp32 attention with a workspace: the (32-query block, head) units are split over key ranges
+    so that small active sets fill the GPU, and a second kernel merges the ranges (the tiny loop's
+    1024- and 512-row steps, a ragged block, a single query row)."""
+    D = 128 * H
+    q, k, v = S.normal(64, (M, D)), S.normal(65, (L, D)), S.normal(66, (L, D))
+    need = cuda_lib.attention_workspace_size(M, L, H, cuda_lib.HSA_F32)
+    assert need > 0
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    o = torch.empty((M, D), device="cuda")
+    cuda_lib.attention(dev(q), dev(k), dev(v), H, o, ws=ws)
+    assert cuda_lib.device_status() == 0
     assert_f32_close(host(o), O.attention(q, k, v))

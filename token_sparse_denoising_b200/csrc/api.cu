@@ -13,7 +13,9 @@ int gemm_f32(const float* A, int M, int K, const float* W, int Nout, const float
 int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, int H, void* O, cudaStream_t st,
                    void* ws, size_t ws_bytes);
 size_t attention_split_bytes(int M, int L, int H);
-int attention_f32(const float* Q, int M, const float* K, const float* V, int L, int H, float* O, cudaStream_t st);
+int attention_f32(const float* Q, int M, const float* K, const float* V, int L, int H, float* O, cudaStream_t st,
+                  void* ws, size_t ws_bytes);
+size_t attention_f32_split_bytes(int M, int L, int H);
 
 static inline unsigned warp_blocks(long long rows) { return (unsigned)((rows * 32 + 255) / 256); }
 static inline size_t esize(int dtype) { return dtype == HSA_BF16 ? 2 : 4; }
@@ -82,7 +84,7 @@ static int attention(const void* q, int M, const void* k, const void* v, int L, 
                      cudaStream_t st, void* ws = nullptr, size_t ws_bytes = 0) {
   if (dtype == HSA_BF16) return attention_bf16(q, M, k, v, L, H, o, st, ws, ws_bytes);
   return attention_f32(static_cast<const float*>(q), M, static_cast<const float*>(k),
-                       static_cast<const float*>(v), L, H, static_cast<float*>(o), st);
+                       static_cast<const float*>(v), L, H, static_cast<float*>(o), st, ws, ws_bytes);
 }
 
 }  // namespace hsa
@@ -147,7 +149,7 @@ extern "C" int hsa_attention(const void* d_q, int M, const void* d_k, const void
 }
 
 extern "C" size_t hsa_attention_workspace_size(int M, int L, int H, int dtype) {
-  return dtype == HSA_BF16 ? attention_split_bytes(M, L, H) : 0;
+  return dtype == HSA_BF16 ? attention_split_bytes(M, L, H) : attention_f32_split_bytes(M, L, H);
 }
 
 extern "C" int hsa_attention_ws(const void* d_q, int M, const void* d_k, const void* d_v, int L, int H, int dtype,

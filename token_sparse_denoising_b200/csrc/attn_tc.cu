@@ -50,6 +50,8 @@ namespace hsa {
 constexpr int kAttnBM = 128;
 constexpr int kAttnBN = 128;
 constexpr int kKSlots = 3;
+// Key ranges of at most this many 128-key tiles run two query tiles per CTA (k_attn_tc<true>)
+constexpr int kTwoQMaxTiles = 8;
 constexpr int kVSlots = 2;
 constexpr int kAttnThreads = 320;                 // 2 control warps + 8 softmax warps
 constexpr int kTileBytes = 128 * 128 * 2;         // one 128 x 128 bf16 operand tile (two 64-column boxes)
@@ -140,15 +142,29 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// kTwoQ: the CTA takes two 128-query tiles of one head (256 queries) and streams each key tile
+// once for both.  Virtual tile t = 2 j + b is key tile j of query tile b, so the parity of a
+// virtual tile is its query tile, and the parity machinery below (S, O and softmax warps per
+// parity, the MMA issue order) runs over 2 nj virtual tiles.  K_j and V_j are loaded once, with
+// the even virtual tile's barriers, and released after the odd virtual tile's QK^T / PV; the
+// parity-1 P barriers count the softmax threads alone (the producer has nothing to add there),
+// and the producer waits for the previous phase of the parity-0 barriers before arriving on them
+// (its ring slots come back only two phases after their last use, which alone would let an
+// arrival land in the phase before its own); the epilogue writes each parity's own rows instead
+// of merging the two.  Used for short key ranges (the cross-attention's
+// context), where filling and draining the pipeline dominates a unit.
+template <bool kTwoQ>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, int M, int L, int H, __nv_bfloat16* __restrict__ O,
               const AttnGrid grid) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int QTILES = kTwoQ ? 2 : 1;                 // query tiles of the CTA
+  constexpr int KS = kTwoQ ? 2 : kKSlots;                // K ring slots (shared memory: 6 tiles either way)
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + kTileBytes;                       // slot s at s * kTileBytes
-  uint8_t* sV = sK + kKSlots * kTileBytes;
+  uint8_t* sK = smem + QTILES * kTileBytes;              // slot s at s * kTileBytes
+  uint8_t* sV = sK + KS * kTileBytes;
   AttnShared* sh = reinterpret_cast<AttnShared*>(sV + kVSlots * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -160,21 +176,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     n_split = grid.s_tail;
     if (n_split > 1) slot = t;
   }
-  const int m0 = (u % grid.QT) * kAttnBM, h = u / grid.QT;
+  const int m0 = (u % grid.QT) * kAttnBM * QTILES, h = u / grid.QT;
   // this CTA's key tiles [j0, j0 + nj): loops, ring slots and parities use the local index
   const int nj_all = (L + kAttnBN - 1) / kAttnBN;
   const int j0 = split * nj_all / n_split;
   const int nj = (split + 1) * nj_all / n_split - j0;
+  const int nt = kTwoQ ? 2 * nj : nj;                    // virtual tiles (key tile x query tile)
+  // key tile of virtual tile t
+  auto key_of = [](int t) { return kTwoQ ? t >> 1 : t; };
 
   if (threadIdx.x == 0) {
     mbar_init(&sh->q_full, 1);
-    for (int s = 0; s < kKSlots; ++s) mbar_init(&sh->k_empty[s], 1);
+    for (int s = 0; s < KS; ++s) mbar_init(&sh->k_empty[s], 1);
     for (int s = 0; s < 2; ++s) mbar_init(&sh->k_full[s], 1);
     for (int s = 0; s < kVSlots; ++s) mbar_init(&sh->v_empty[s], 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh->s_full[b], 1);
-      mbar_init(&sh->p_full[b][0], 129);
-      mbar_init(&sh->p_full[b][1], 129);
+      // the softmax threads, plus one producer arrival (with the bytes of V_j / the next K) where
+      // the producer has something to deliver: every tile, or the even virtual tiles of kTwoQ
+      const uint32_t n_arrive = (kTwoQ && b == 1) ? 128 : 129;
+      mbar_init(&sh->p_full[b][0], n_arrive);
+      mbar_init(&sh->p_full[b][1], n_arrive);
     }
     mbar_init(&sh->o_done, 1);
     fence_mbar_init();
@@ -196,14 +218,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int x0 = h * 128;
     const bool leader = elect_one();
     if (leader) {
-      mbar_expect_tx(&sh->q_full, kTileBytes);
-      tma_load_2d(sQ, &tmQ, &sh->q_full, x0, m0);
-      tma_load_2d(sQ + kTileBytes / 2, &tmQ, &sh->q_full, x0 + 64, m0);
+      mbar_expect_tx(&sh->q_full, QTILES * kTileBytes);
+#pragma unroll
+      for (int qt = 0; qt < QTILES; ++qt) {
+        tma_load_2d(sQ + qt * kTileBytes, &tmQ, &sh->q_full, x0, m0 + qt * kAttnBM);
+        tma_load_2d(sQ + qt * kTileBytes + kTileBytes / 2, &tmQ, &sh->q_full, x0 + 64, m0 + qt * kAttnBM);
+      }
     }
-    // K_j into its ring slot, completing on `bar`
+    // K of key tile j into its ring slot, completing on `bar`
     auto load_k = [&](int j, uint64_t* bar) -> bool {
-      const int sk = j % kKSlots;
-      const bool ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->k_empty[sk], ((j / kKSlots) & 1) ^ 1), 0);
+      const int sk = j % KS;
+      const bool ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->k_empty[sk], ((j / KS) & 1) ^ 1), 0);
       __syncwarp();
       if (ok && leader) {
         uint8_t* k = sK + sk * kTileBytes;
@@ -214,21 +239,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       return ok;
     };
     bool ok = load_k(0, &sh->k_full[0]);
-    if (ok && nj > 1) ok = load_k(1, &sh->k_full[1]);
+    if (!kTwoQ && ok && nj > 1) ok = load_k(1, &sh->k_full[1]);
     static_assert(kVSlots == 2, "V slot j % 2 is also the parity of tile j");
-    for (int j = 0; ok && j < nj; ++j) {
-      const int b = j & 1;
-      ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->v_empty[b], ((j >> 1) & 1) ^ 1), 0);
+    // kTwoQ: only the even virtual tiles (t = 2 j) have something to deliver -- V_j, and the K of
+    // QK^T(t + 2) = K_{j+1}; the odd ones read the same V_j and issue QK^T with K_{j+1} after the
+    // even tile's barriers completed, so the producer skips them
+    for (int t = 0; ok && t < nt; t += kTwoQ ? 2 : 1) {
+      const int b = t & 1, j = key_of(t), sv = j & 1;
+      ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->v_empty[sv], ((j >> 1) & 1) ^ 1), 0);
       __syncwarp();
+      if (kTwoQ && ok && j > 0) {
+        // a ring slot comes back two phases after its last use here, so wait for the previous
+        // phase of both barriers before arriving on them: an arrival is never counted early
+        ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->p_full[0][0], (j - 1) & 1), 0);
+        if (ok) ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->p_full[0][1], (j - 1) & 1), 0);
+        __syncwarp();
+      }
       if (!ok) break;
       if (leader) {
-        uint8_t* v = sV + b * kTileBytes;
+        uint8_t* v = sV + sv * kTileBytes;
         mbar_expect_tx(&sh->p_full[b][0], kTileBytes);
         tma_load_2d(v, &tmV, &sh->p_full[b][0], x0, (j0 + j) * kAttnBN);
         tma_load_2d(v + kTileBytes / 2, &tmV, &sh->p_full[b][0], x0 + 64, (j0 + j) * kAttnBN);
       }
-      if (j + 2 < nj) {
-        ok = load_k(j + 2, &sh->p_full[b][1]);
+      if (t + 2 < nt) {
+        ok = load_k(key_of(t + 2), &sh->p_full[b][1]);
       } else {
         if (leader) mbar_arrive(&sh->p_full[b][1]);
         __syncwarp();
@@ -250,29 +285,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       return r;
     };
-    // QK^T of tile j; tiles 0 and 1 wait for their K here, later ones through p_full
-    auto issue_qk = [&](int j) -> bool {
-      const int sk = j % kKSlots, b = j & 1;
-      if (j < 2 && !wait_all(&sh->k_full[j], 0)) return false;
+    // QK^T of virtual tile t; the first two wait for their K here, later ones through p_full
+    auto issue_qk = [&](int t) -> bool {
+      const int j = key_of(t), sk = j % KS, b = t & 1;
+      if (t < 2 && !wait_all(&sh->k_full[kTwoQ ? 0 : t], 0)) return false;
       tc_fence_after();
       const uint64_t kd = k_desc + (uint64_t)((sk * kTileBytes) >> 4);
+      const uint64_t qd = q_desc + (uint64_t)(((kTwoQ ? b : 0) * kTileBytes) >> 4);
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
-          umma_ss(tm + kColS + b * 128, q_desc + off, kd + off, idesc_s, kk > 0);
+          umma_ss(tm + kColS + b * 128, qd + off, kd + off, idesc_s, kk > 0);
         }
         umma_commit(&sh->s_full[b]);
-        umma_commit(&sh->k_empty[sk]);        // K_j is free once S_j is computed
+        // K_j is free once every S it feeds is computed
+        if (!kTwoQ || b == 1) umma_commit(&sh->k_empty[sk]);
       }
       __syncwarp();
       return true;
     };
     bool ok = wait_all(&sh->q_full, 0);
     if (ok) ok = issue_qk(0);
-    if (ok && nj > 1) ok = issue_qk(1);
-    for (int j = 0; ok && j < nj; ++j) {
-      const int b = j & 1, sv = j % kVSlots;
+    if (ok && nt > 1) ok = issue_qk(1);
+    for (int t = 0; ok && t < nt; ++t) {
+      const int b = t & 1, j = key_of(t), sv = j % kVSlots;
       const uint64_t vd = v_desc + (uint64_t)((sv * kTileBytes) >> 4);
 
       // PV half by half of the keys: the first starts while the softmax warps are still
@@ -280,22 +317,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool got = true;
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        // half 0 also brings V_j, half 1 also K_{j+2}
-        if (!wait_all(&sh->p_full[b][q], (j >> 1) & 1)) { got = false; break; }
+        // half 0 also brings V_j, half 1 also the K of QK^T(t + 2) (even virtual tiles only with kTwoQ)
+        if (!wait_all(&sh->p_full[b][q], (t >> 1) & 1)) { got = false; break; }
         tc_fence_after();
         if (leader) {
 #pragma unroll
           for (int kk = q * 4; kk < q * 4 + 4; ++kk) {
             // V tile: key rows of 128 B (64 channels) per box; 16 keys = two 1024-byte atoms
             umma_ts(tm + kColO + b * 128, tm + kColS + b * 128 + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), idesc_o,
-                    (j >= 2 || kk > 0));
+                    (t >= 2 || kk > 0));
           }
-          if (q == 1) umma_commit(&sh->v_empty[sv]);
+          // V_j is free once every PV that reads it is issued
+          if (q == 1 && (!kTwoQ || b == 1)) umma_commit(&sh->v_empty[sv]);
         }
         __syncwarp();
       }
       if (!got) break;
-      if (j + 2 < nj) ok = issue_qk(j + 2);   // overwrites S_b (P_j) after PV_j in issue order
+      if (t + 2 < nt) ok = issue_qk(t + 2);   // overwrites S_b (P_t) after PV_t in issue order
     }
     if (leader) umma_commit(&sh->o_done);   // every MMA of this CTA, both O accumulators
     __syncwarp();
@@ -308,8 +346,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t s_col = lane_base + kColS + par * 128, o_col = lane_base + kColO + par * 128;
     const float sc = 0.12751743074680484f;          // log2(e) / sqrt(128)
     float m = -INFINITY, l = 0.f;
-    for (int j = par; j < nj; j += 2) {
-      mbar_wait(&sh->s_full[par], (j >> 1) & 1);
+    for (int t = par; t < nt; t += 2) {
+      const int j = key_of(t);
+      mbar_wait(&sh->s_full[par], (t >> 1) & 1);
       __syncwarp();
       tc_fence_after();
       uint32_t sr[128];
@@ -336,7 +375,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // after P is stored, when the S registers are free
       bool need = false;
       float corr = 1.0f;
-      if (j == par) {
+      if (t == par) {
         m = m_tile;
       } else if (m_tile > m + 8.0f) {
         need = true;
@@ -393,6 +432,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(&sh->p_full[par][1]);
     }
     // ---------------------------------------------------------------- epilogue
+    if constexpr (kTwoQ) {
+      // each parity holds its own query tile: O_par / l for rows m0 + 128 par + row
+      mbar_wait(&sh->o_done, 0);
+      __syncwarp();
+      tc_fence_after();
+      const int grow = m0 + par * kAttnBM + row;
+      const float inv_l = 1.0f / l;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        __syncwarp();
+        tmem_ld32(o_col + c * 32, o);
+        tmem_ld_wait();
+        if (grow < M) {
+          __nv_bfloat16* dst = O + (size_t)grow * (H * 128) + h * 128 + c * 32;
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 pk4;
+            pk4.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+            pk4.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+            pk4.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+            pk4.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(dst + e) = pk4;
+          }
+        }
+      }
+    } else {
     // merge the two parities; parity 1 has tiles only when nj >= 2
     sh->xm[par][row] = m;
     sh->xl[par][row] = l;
@@ -463,6 +529,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
     }
+    }  // two-parity merge
   }
 
   tc_fence_before();
@@ -538,6 +605,7 @@ size_t tail_split_bytes(const TailSplit& p) {
 
 size_t attention_split_bytes(int M, int L, int H) {
   if (M <= 0 || L <= 0 || H <= 0) return 0;
+  if ((L + kAttnBN - 1) / kAttnBN <= kTwoQMaxTiles && M > kAttnBM) return 0;   // two-query-tile CTAs: no split
   const int QT = (M + kAttnBM - 1) / kAttnBM;
   return tail_split_bytes(plan_tail(QT * H, (L + kAttnBN - 1) / kAttnBN, num_sms()));
 }
@@ -558,13 +626,26 @@ int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, in
   if (rc) return rc;
   static PerContextOnce attr;
   rc = attr.ensure([](void**) {
-    if (cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_attn_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(k_attn_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess)
       return check_launch("attention: shared-memory attribute");
     return (int)HSA_OK;
   });
   if (rc) return rc;
+  const int nj_all = (L + kAttnBN - 1) / kAttnBN;
+  if (nj_all <= kTwoQMaxTiles && M > kAttnBM) {
+    // short key range: two query tiles per CTA share every K/V tile, no key-range split
+    const int QT2 = (M + 2 * kAttnBM - 1) / (2 * kAttnBM);
+    AttnGrid g{QT2, QT2 * H, 1, nullptr, nullptr};
+    ScopedTiming timing(HSA_KCLASS_ATTENTION, st);
+    k_attn_tc<true><<<QT2 * H, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, M, L, H,
+                                                               reinterpret_cast<__nv_bfloat16*>(O), g);
+    count_launch(1);
+    return check_launch("attn_tc (two query tiles) launch");
+  }
   const int QT = (M + kAttnBM - 1) / kAttnBM, U = QT * H;
-  TailSplit ts = plan_tail(U, (L + kAttnBN - 1) / kAttnBN, num_sms());
+  TailSplit ts = plan_tail(U, nj_all, num_sms());
   const size_t need = tail_split_bytes(ts);
   if (need == 0 || !ws || ws_bytes < need || !aligned16(ws)) ts = TailSplit{U, 1, 0};
   AttnGrid g{QT, ts.u_full, ts.s_tail, nullptr, nullptr};
@@ -575,7 +656,8 @@ int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, in
   }
   ScopedTiming timing(HSA_KCLASS_ATTENTION, st);
   const int ctas = ts.u_full + ts.n_tail * ts.s_tail;
-  k_attn_tc<<<ctas, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, M, L, H, reinterpret_cast<__nv_bfloat16*>(O), g);
+  k_attn_tc<false><<<ctas, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, M, L, H, reinterpret_cast<__nv_bfloat16*>(O),
+                                                          g);
   count_launch(1);
   if (ts.s_tail > 1) {
     rc = check_launch("attn_tc launch");
