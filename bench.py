@@ -56,10 +56,11 @@ def parse():
     p.add_argument("--no-configs", action="store_true",
                    help="skip the other workloads measured beside the headline (tiny loop, 30-block loop, "
                         "Wan-14B block, attention and Euler sweeps)")
-    p.add_argument("--mode", choices=["step", "loop", "sweep", "wan14", "tiny"], default="step",
+    p.add_argument("--mode", choices=["step", "loop", "sweep", "wan14", "tiny", "headpar"], default="step",
                    help="step: the headline line; loop: 30-block Wan-1.3B loop, HSA vs uniform 40 steps; "
                         "sweep: attention + Euler kernel sweep; wan14: Wan-14B block active-fraction sweep; "
-                        "tiny: the fp32 parity workload as a whole run")
+                        "tiny: the fp32 parity workload as a whole run; headpar: one Wan-14B block split by "
+                        "heads over the ranks (NCCL between the phases), |A|/N = 1")
     return p.parse_args()
 
 
@@ -532,6 +533,20 @@ def measure_sweep(reps: int = 5):
             tf = 4.0 * M * N * 128 * 12 / (ms * 1e-3) / 1e12
             res["attention"].append({"N": N, "frac": f, "M": M, "ms": round(ms, 4), "tflops": round(tf, 1),
                                      "frac_of_burst": round(tf / peak_burst, 3)})
+        if N == 32760:
+            # the oracle's attention of 8 query rows over the same keys (copied to the host)
+            from oracle import hsa_oracle as O
+            kh, vh_ = k.float().cpu().numpy().astype(np.float64), v.float().cpu().numpy().astype(np.float64)
+            qh = S.device_normal(gen, (8, 1536), 1.0, True, "cuda").float().cpu().numpy().astype(np.float64)
+            t0 = time.perf_counter()
+            O.attention(qh, kh, vh_)
+            row_ms = (time.perf_counter() - t0) * 1e3 / 8
+            res["oracle"] = {"kind": "oracle", "cores": blas_threads(), "N": N,
+                             "measured_per_unit_ms": {"query_row_ms": round(row_ms, 3)},
+                             "value_ms_full": round(row_ms * N, 1),
+                             "sample": f"fp64 numpy oracle attention of 8 query rows over {N} keys, 12 heads; "
+                                       f"value = query_row_ms x {N} (the |A|/N = 1 launch)"}
+            del kh, vh_
         del k, v
     # the cross-attention shape: every active query against the 512-row text context
     M, L = S.WAN13_GRID.N, S.WAN13_BLOCK.ctx_len
@@ -598,9 +613,12 @@ def measure_sweep(reps: int = 5):
     return res
 
 
-def measure_wan14(patterns=("contiguous", "scattered"), reps: int = 3):
+def measure_wan14(patterns=("contiguous", "scattered"), reps: int = 3, with_oracle: bool = False):
     """Wan-14B block (D=5120, 40 heads, FFN 13824, no context) at |A|/N in {1, .5, .25, .125}:
-    layer-step ms for contiguous and/or scattered active sets.  Weights drawn on the device."""
+    layer-step ms for contiguous and/or scattered active sets.  Weights drawn on the device.  With
+    `with_oracle`, the oracle on the same weights and inputs (copied to the host) on a sample: the
+    q/k/v projections of 128 tokens and attention over all N cache rows + O-projection + FFN of 4
+    query rows, extrapolated to the |A|/N = 1 step."""
     import torch
     from token_sparse_denoising_b200 import hsa
     hsa.load()
@@ -630,9 +648,35 @@ def measure_wan14(patterns=("contiguous", "scattered"), reps: int = 3):
             res["points"].append({"frac": f, "pattern": pattern, "M": M, "ms": round(ms, 3), "tflops": round(tf, 1),
                                   "frac_of_burst": round(tf / peak_burst, 3)})
     assert hsa.device_status() == 0
+    if with_oracle:
+        res["oracle"] = _oracle_block_sample(w, x, kc, vc, S.token_positions(grid), n_tok=128, n_rows=4)
     del w, kc, vc, x, ws, xA
     torch.cuda.empty_cache()
     return res
+
+
+def _oracle_block_sample(w, x, kc, vc, pos, n_tok: int, n_rows: int):
+    """The fp64 oracle on a sample of one |A|/N = 1 step of a block whose inputs live on the device
+    (pulled to the host first, not timed): per-token and per-query-row times and the extrapolation."""
+    from oracle import hsa_oracle as O
+    N, D = x.shape
+    host = lambda t: t.float().cpu().numpy()
+    bw = S.BlockWeights(**{k: host(w.t[k]) for k in ("w_qkv", "b_qkv", "g_q", "g_k", "w_o", "b_o", "w_1", "b_1",
+                                                       "w_2", "b_2", "mod")})
+    X = host(x[:: N // n_tok][:n_tok]).astype(np.float64)
+    tok = np.arange(0, N, N // n_tok)[:n_tok]
+    Kc, Vc = host(kc).astype(np.float64), host(vc).astype(np.float64)
+    t0 = time.perf_counter()
+    q, k, v = O.qkv_projection(bw, X, pos[tok])
+    t1 = time.perf_counter()
+    O.block_tail(bw, X[:n_rows], O.attention(q[:n_rows], Kc, Vc), None)
+    t2 = time.perf_counter()
+    tok_ms, row_ms = (t1 - t0) * 1e3 / n_tok, (t2 - t1) * 1e3 / n_rows
+    return {"kind": "oracle", "cores": blas_threads(), "value_ms_full_step": round((tok_ms + row_ms) * N, 1),
+            "measured_per_unit_ms": {"token_ms": round(tok_ms, 4), "query_row_ms": round(row_ms, 3)},
+            "sample": f"fp64 numpy oracle: q/k/v projections of {n_tok} tokens, attention over all {N} cache rows "
+                      f"+ O-projection + FFN of {n_rows} query rows; value = (token_ms + query_row_ms) x {N}, "
+                      f"the |A|/N = 1 step"}
 
 
 def run_loop(args):
@@ -651,10 +695,52 @@ def run_wan14(args):
     return {"mode": "wan14", **measure_wan14()}
 
 
+def run_headpar(args, rank, world, barrier, allmax, dist):
+    """One Wan-14B-shaped block (N = 32760, D = 5120, 40 heads, FFN 13824, every token active) split
+    by heads over the `world` ranks: rank r holds 40/world heads (their q/k/v rows, KV cache columns
+    and W_o columns), 13824/world FFN columns and 1/world of the residual rows; all-gather /
+    all-reduce / reduce-scatter over NCCL between the phases.  ms per block step, max over ranks."""
+    import torch
+    from token_sparse_denoising_b200 import hsa, sharded
+    hsa.load()
+    grid, shape = S.WAN13_GRID, S.WAN14_BLOCK
+    N, D = grid.N, shape.D
+    dev = torch.device("cuda", torch.cuda.current_device())
+    shard = sharded.HeadShard(rank, world, shape.H, shape.F, N)
+    bw = S.block_weights_on_device(4, shape, True, dev)        # the same draws on every rank
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(14)
+    kc = S.device_normal(gen, (N, D), 1.0, True, dev)
+    vc = S.device_normal(gen, (N, D), 1.0, True, dev)
+    x = S.device_normal(gen, (N, D), 1.0, False, dev)
+    blk = sharded.HeadParallelBlock(bw, shard, N, dev, cache_init=(kc, vc))
+    del bw, kc, vc
+    torch.cuda.empty_cache()
+    idx = torch.arange(N, dtype=torch.int32, device=dev)
+    pos = torch.from_numpy(S.token_positions(grid)).to(dev)
+    if dist is None:
+        step = lambda: sharded.EmulatedGroup.run([blk.step(x, idx, pos)])
+    else:
+        step = lambda: sharded.run_collectives(blk.step(x, idx, pos), dist)
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    ms = allmax(time_device(step, steps, barrier)) / steps
+    assert hsa.device_status() == 0
+    flops = 4.0 * N * N * 128 * shape.H + 2.0 * N * (3 * D * D + D * D + 2 * D * shape.F)
+    return {"mode": "headpar", "metric": "Wan-14B block step ms, heads split over the ranks", "value": round(ms, 3),
+            "unit": "ms", "n_gpus": world, "steps": steps, "higher_is_better": False, "scaling": "strong",
+            "config": {"workload": "wan14b-block N=32760 D=5120 H=40 F=13824 |A|/N=1",
+                       "parallelism": f"heads/{world} per rank, NCCL all-gather + all-reduce + reduce-scatter"},
+            "tflops_aggregate": round(flops / (ms * 1e-3) / 1e12, 1)}
+
+
 def measure_configs():
     """The other workloads, measured beside the headline step on the same GPU in the same run."""
     t0 = time.perf_counter()
-    out = {"attention_euler_sweep": measure_sweep(), "wan14_block": measure_wan14(patterns=("contiguous",)),
+    out = {"attention_euler_sweep": measure_sweep(),
+           "wan14_block": measure_wan14(patterns=("contiguous",), with_oracle=True),
            "tiny_fp32_loop": measure_tiny(with_oracle=True), "wan13_loop": measure_loop(graph=False)}
     out["wall_s"] = round(time.perf_counter() - t0, 1)
     return out
@@ -806,6 +892,23 @@ def main():
 
     import torch
     torch.cuda.set_device(local)
+    if args.mode == "headpar":
+        dist = None
+        if world > 1 or "RANK" in os.environ:          # under torchrun: NCCL even for one rank
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        barrier, allmax = collectives(dist, "cuda")
+        try:
+            out = run_headpar(args, rank, world, barrier, allmax, dist)
+        finally:
+            if dist is not None:
+                dist.barrier()
+                dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        return 0
     if args.mode != "step":
         if rank == 0:
             fn = {"loop": run_loop, "sweep": run_sweep, "wan14": run_wan14, "tiny": run_tiny}[args.mode]
@@ -831,6 +934,15 @@ def main():
             out["configs"] = measure_configs()
         if world == 1 and not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_baseline(synthetic_inputs())
+            loop = out.get("configs", {}).get("wan13_loop")
+            if loop:
+                u = out["cpu_baseline"]["measured_per_unit_ms"]
+                blocks = S.WAN13_LOOP.n_blocks
+                for name in ("hsa", "uniform"):
+                    loop[name]["oracle_ms_estimate"] = round(
+                        loop[name]["token_steps"] * (u["token_ms"] + u["query_row_ms"]) * blocks, 0)
+                loop["oracle_note"] = ("estimate, not a run: the oracle's measured per-token and per-query-row "
+                                       f"costs of one Wan-1.3B block x {blocks} blocks x the run's token-steps")
         print(json.dumps(out), flush=True)
     return 0
 
