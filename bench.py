@@ -56,11 +56,12 @@ def parse():
     p.add_argument("--no-configs", action="store_true",
                    help="skip the other workloads measured beside the headline (tiny loop, 30-block loop, "
                         "Wan-14B block, attention and Euler sweeps)")
-    p.add_argument("--mode", choices=["step", "loop", "sweep", "wan14", "tiny", "headpar"], default="step",
+    p.add_argument("--mode", choices=["step", "loop", "sweep", "wan14", "tiny", "headpar", "cross"], default="step",
                    help="step: the headline line; loop: 30-block Wan-1.3B loop, HSA vs uniform 40 steps; "
                         "sweep: attention + Euler kernel sweep; wan14: Wan-14B block active-fraction sweep; "
                         "tiny: the fp32 parity workload as a whole run; headpar: one Wan-14B block split by "
-                        "heads over the ranks (NCCL between the phases), |A|/N = 1")
+                        "heads over the ranks (NCCL between the phases), |A|/N = 1; cross: the "
+                        "cross-attention shape alone (32760 queries x 512 context rows)")
     return p.parse_args()
 
 
@@ -90,12 +91,50 @@ def synthetic_inputs():
 # ---------------------------------------------------------------- clocks during the timed region
 
 class ClockSampler:
-    """nvidia-smi polled every 50 ms from before the warm-up; stop() keeps the samples whose
+    """SM clock, instantaneous power and clock-event reasons, sampled from before the warm-up:
+    NVML read every 10 ms on a host thread (read-only queries), and nvidia-smi every 50 ms beside
+    it as a cross-check (alone where NVML cannot be used).  stop() keeps the samples whose
     timestamps fall inside the timed region (host clock window set by mark_start / mark_end)."""
 
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
     def __init__(self, index: int):
-        self.path = tempfile.mktemp(suffix=".csv")
         self.t0 = self.t1 = None
+        self.rows = []                          # (time, sm MHz, max MHz, power W, [reasons])
+        self.proc = self.thread = None
+        self.stop_flag = False
+        try:
+            import threading
+            import pynvml as N
+            import torch
+            N.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(index).uuid)
+            self.h = N.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+            bits = {"hw_slowdown": N.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": N.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": N.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": N.nvmlClocksEventReasonSwPowerCap}
+            max_mhz = float(N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM))
+
+            def poll():
+                while not self.stop_flag:
+                    r = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    pw = N.nvmlDeviceGetFieldValues(self.h, [N.NVML_FI_DEV_POWER_INSTANT])[0]
+                    self.rows.append((time.time(), float(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM)),
+                                      max_mhz, pw.value.uiVal / 1000.0 if pw.nvmlReturn == 0 else float("nan"),
+                                      [n for n in self.NAMES if r & bits[n]]))
+                    time.sleep(0.01)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.thread = None
+        self._start_smi(index)
+        self.source = "NVML every 10 ms" if self.thread is not None else "nvidia-smi every 50 ms"
+        time.sleep(0.2)                        # sampling runs before the work starts
+
+    def _start_smi(self, index):
+        self.path = tempfile.mktemp(suffix=".csv")
         q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw.instant,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -103,7 +142,7 @@ class ClockSampler:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}",
                                           "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-            time.sleep(0.5)                    # let nvidia-smi start sampling before the work
+            time.sleep(0.3)
         except OSError:
             self.proc = None
 
@@ -113,14 +152,13 @@ class ClockSampler:
     def mark_end(self):
         self.t1 = time.time()
 
-    def stop(self):
+    def _smi_rows(self):
         import datetime
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return []
         self.proc.terminate()
         self.proc.wait(timeout=10)
         rows = []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             f = [v.strip() for v in line.split(",")]
             if len(f) < 10:
@@ -128,10 +166,13 @@ class ClockSampler:
             try:
                 ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
                 rows.append((ts, float(f[2]), float(f[3]), float(f[4]),
-                             [n for n, v in zip(names, f[6:10]) if v.lower() == "active"]))
+                             [n for n, v in zip(self.NAMES, f[6:10]) if v.lower() == "active"]))
             except ValueError:
                 continue
         os.unlink(self.path)
+        return rows
+
+    def _select(self, rows):
         window = "timed region"
         sel = [r for r in rows if self.t0 is not None and self.t0 <= r[0] <= self.t1]
         if len(sel) < 2:                        # a very short timed region: add the warm-up just before it
@@ -139,11 +180,31 @@ class ClockSampler:
             sel = [r for r in rows if self.t0 is not None and self.t0 - 1.0 <= r[0] <= self.t1]
         if not sel:
             window, sel = "whole run", rows
+        return window, sel
+
+    def stop(self):
+        smi = self._smi_rows()
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            rows = list(self.rows)
+        elif smi:
+            rows = smi
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        window, sel = self._select(rows)
         reasons = sorted({n for r in sel for n in r[4]})
-        return {"sm_mhz": statistics.median(r[1] for r in sel) if sel else None,
-                "sm_max_mhz": sel[-1][2] if sel else None, "reasons": reasons,
-                "power_w_median": statistics.median(r[3] for r in sel) if sel else None,
-                "samples": len(sel), "window": window}
+        out = {"sm_mhz": statistics.median(r[1] for r in sel) if sel else None,
+               "sm_max_mhz": sel[-1][2] if sel else None, "reasons": reasons,
+               "power_w_median": round(statistics.median(r[3] for r in sel), 1) if sel else None,
+               "samples": len(sel), "window": window, "source": self.source}
+        if self.thread is not None and smi:
+            w2, s2 = self._select(smi)
+            out["nvidia_smi"] = {"sm_mhz": statistics.median(r[1] for r in s2),
+                                 "power_w_median": statistics.median(r[3] for r in s2),
+                                 "reasons": sorted({n for r in s2 for n in r[4]}), "samples": len(s2),
+                                 "window": w2}
+        return out
 
 
 # ---------------------------------------------------------------- the CUDA path
@@ -508,6 +569,29 @@ def measure_tiny(with_oracle: bool = True, reps: int = 5):
     return out
 
 
+def measure_cross(reps: int = 20, gen=None):
+    """The cross-attention shape alone: every active query of the Wan-1.3B block (32760) against
+    the 512-row text context, 12 heads, bf16; two warm-up launches, then `reps` timed back to back."""
+    import torch
+    from token_sparse_denoising_b200 import hsa
+    hsa.load()
+    _, peak_burst, _, _ = load_peaks()
+    if gen is None:
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(5)
+    M, L = S.WAN13_GRID.N, S.WAN13_BLOCK.ctx_len
+    k = S.device_normal(gen, (L, 1536), 1.0, True, "cuda")
+    v = S.device_normal(gen, (L, 1536), 1.0, True, "cuda")
+    q = S.device_normal(gen, (M, 1536), 1.0, True, "cuda")
+    o = torch.empty_like(q)
+    for _ in range(2):
+        hsa.attention(q, k, v, 12, o)
+    ms = time_device(lambda: hsa.attention(q, k, v, 12, o), reps, lambda: None) / reps
+    tf = 4.0 * M * L * 128 * 12 / (ms * 1e-3) / 1e12
+    assert hsa.device_status() == 0
+    return {"M": M, "L": L, "H": 12, "ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_burst": round(tf / peak_burst, 3)}
+
+
 def measure_sweep(reps: int = 5):
     """Attention at N in {8190, 32760, 75600} x |A|/N in {1, .5, .25, .125} (12 heads, bf16 Q/K/V
     N(0,1)) and the Euler update on N x 64 fp32 latents with the L2 flushed before each launch."""
@@ -548,19 +632,7 @@ def measure_sweep(reps: int = 5):
                                        f"value = query_row_ms x {N} (the |A|/N = 1 launch)"}
             del kh, vh_
         del k, v
-    # the cross-attention shape: every active query against the 512-row text context
-    M, L = S.WAN13_GRID.N, S.WAN13_BLOCK.ctx_len
-    k = S.device_normal(gen, (L, 1536), 1.0, True, "cuda")
-    v = S.device_normal(gen, (L, 1536), 1.0, True, "cuda")
-    q = S.device_normal(gen, (M, 1536), 1.0, True, "cuda")
-    o = torch.empty_like(q)
-    for _ in range(2):
-        hsa.attention(q, k, v, 12, o)
-    ms = time_device(lambda: hsa.attention(q, k, v, 12, o), 4 * reps, lambda: None) / (4 * reps)
-    tf = 4.0 * M * L * 128 * 12 / (ms * 1e-3) / 1e12
-    res["cross_attention"] = {"M": M, "L": L, "H": 12, "ms": round(ms, 4), "tflops": round(tf, 1),
-                              "frac_of_burst": round(tf / peak_burst, 3)}
-    del q, k, v, o
+    res["cross_attention"] = measure_cross(4 * reps, gen)
     flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda")      # 256 MB > L2: evicts between launches
     flush_r = torch.zeros(256 * 1024 * 1024 // 4, device="cuda")
     for N in (8190, 32760, 75600):
@@ -585,27 +657,49 @@ def measure_sweep(reps: int = 5):
                  "l2": "written (256 MB) then read (256 MB) before each launch, so no dirty line of the flush is "
                        "written back inside the timed launch"}
         del x, vh
-        # back to back, as in a run: launches over distinct (x, v_hat) sets whose total is >= 2x L2
+        # back to back, as in a recorded run: the launches over distinct (x, v_hat) sets, whose total
+        # is >= 2x L2, recorded as one CUDA graph (the host's per-call cost is then outside the
+        # interval), and the same launches issued one by one from Python for comparison
         sets = max(2, (512 << 20) // (8 * N * 64))
         xs = [torch.randn((N, 64), device="cuda", generator=gen) for _ in range(sets)]
         vs = [torch.randn((N, 64), device="cuda", generator=gen) for _ in range(sets)]
+
+        def issue():
+            for k in range(sets):
+                hsa.euler_update(xs[k], vs[k], None, None, -0.025)
+
         for _ in range(2):
-            for k in range(sets):
-                hsa.euler_update(xs[k], vs[k], None, None, -0.025)
-        bt = []
-        for _ in range(5):
-            a, b = _events()
-            a.record()
-            for k in range(sets):
-                hsa.euler_update(xs[k], vs[k], None, None, -0.025)
-            b.record()
-            b.synchronize()
-            bt.append(a.elapsed_time(b) / sets)
-        ms_b = statistics.median(bt)
+            issue()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=side):
+                issue()
+        torch.cuda.current_stream().wait_stream(side)
+        for _ in range(2):
+            graph.replay()
+
+        def per_launch(fn):
+            out = []
+            for _ in range(5):
+                a, b = _events()
+                a.record()
+                fn()
+                b.record()
+                b.synchronize()
+                out.append(a.elapsed_time(b) / sets)
+            return statistics.median(out)
+
+        ms_b = per_launch(graph.replay)
+        ms_e = per_launch(issue)
+        del graph
         gbs_b = 12 * N * 64 / (ms_b * 1e-3) / 1e9
         entry["back_to_back"] = {"us_per_launch": round(ms_b * 1e3, 2), "gbs": round(gbs_b, 1),
                                  "frac_of_hbm": round(gbs_b / hbm, 3), "sets": sets,
-                                 "working_set_mb": round(sets * 8 * N * 64 / 1e6, 1)}
+                                 "working_set_mb": round(sets * 8 * N * 64 / 1e6, 1),
+                                 "launch": "one CUDA graph of the launches",
+                                 "issued_from_python_us_per_launch": round(ms_e * 1e3, 2)}
         res["euler"].append(entry)
         del xs, vs
     del flush, flush_r
@@ -911,7 +1005,8 @@ def main():
         return 0
     if args.mode != "step":
         if rank == 0:
-            fn = {"loop": run_loop, "sweep": run_sweep, "wan14": run_wan14, "tiny": run_tiny}[args.mode]
+            fn = {"loop": run_loop, "sweep": run_sweep, "wan14": run_wan14, "tiny": run_tiny,
+                  "cross": lambda a: {"mode": "cross", **measure_cross()}}[args.mode]
             print(json.dumps(fn(args)), flush=True)
         return 0
     dist = None

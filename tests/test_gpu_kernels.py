@@ -169,10 +169,13 @@ def test_linear_f32(cuda_lib, M, K, Nout, epi):
 # ------------------------------------------------------------------ §2.2 attention
 
 @pytest.mark.parametrize("M,L,H,qscale", [(200, 1000, 2, 1.0), (128, 128, 1, 1.0), (1, 1, 1, 1.0),
-                                          (257, 300, 3, 4.0), (64, 4000, 2, 1.0),
-                                          # two key tiles: each parity has one tile and no tile j+2
-                                          (130, 256, 2, 1.0), (100, 129, 1, 4.0)])
+                                          (257, 300, 3, 4.0), (130, 256, 2, 1.0), (100, 129, 1, 4.0),
+                                          # more than 8 key tiles: the two-parity kernel
+                                          (64, 4000, 2, 1.0), (130, 1100, 2, 1.0), (257, 1153, 3, 4.0),
+                                          (1, 1025, 1, 1.0), (128, 1152, 1, 1.0)])
 def test_attention_bf16(cuda_lib, M, L, H, qscale):
+    """Key ranges of at most 8 tiles (1024 keys) run the one-parity kernel, longer ones the
+    two-parity kernel: ragged query and key tiles of both, one query row, one key."""
     D = 128 * H
     q = S.normal(31, (M, D), qscale, True)
     k, v = S.normal(32, (L, D), 1.0, True), S.normal(33, (L, D), 1.0, True)
@@ -182,13 +185,15 @@ def test_attention_bf16(cuda_lib, M, L, H, qscale):
     assert_bf16_close(host(o), O.attention(q, k, v), "attention")
 
 
-def test_attention_rescale_across_tiles(cuda_lib):
-    """Logits that jump in a late key tile force the lazy O rescale."""
-    M, L, H = 130, 700, 1
+@pytest.mark.parametrize("L", [700, 1500])
+def test_attention_rescale_across_tiles(cuda_lib, L):
+    """Logits that jump in a late key tile force the lazy O rescale (one-parity kernel at 700
+    keys, two-parity kernel at 1500)."""
+    M, H = 130, 1
     q = S.normal(41, (M, 128), 1.0, True)
     k = S.normal(42, (L, 128), 0.3, True)
     v = S.normal(43, (L, 128), 1.0, True)
-    k[600:610] = S.round_bf16(np.repeat(q[:1] * 0.9, 10, 0))   # large logits for rows like q[0] late
+    k[L - 100:L - 90] = S.round_bf16(np.repeat(q[:1] * 0.9, 10, 0))   # large logits for rows like q[0] late
     k[300] = S.round_bf16(q[5] * 0.7)
     o = torch.empty((M, 128), dtype=torch.bfloat16, device="cuda")
     cuda_lib.attention(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), H, o)
@@ -233,12 +238,14 @@ def test_attention_split_tail_matches_oracle(cuda_lib, M, L, H):
 
 
 @pytest.mark.parametrize("M,L,H", [(256, 512, 12), (300, 16, 2), (200, 300, 2), (2000, 1000, 3), (129, 1024, 1),
-                                   (640, 129, 2)])
-def test_attention_two_query_tiles(cuda_lib, M, L, H):
-    """Key ranges of at most 8 tiles (the cross-attention's context) run two query tiles per CTA,
-    each key tile loaded once for both: exact multiples of 256 queries, a ragged second query
-    tile (300, 200, 2000 rows; 129 rows: a pair with a single real row), a single ragged key tile
-    (16 keys), the largest range that takes this path (1024 keys) and a ragged 129-key range."""
+                                   (640, 129, 2), (100, 512, 2), (1, 64, 1), (4096, 1024, 4), (40000, 64, 1),
+                                   (20000, 300, 3)])
+def test_attention_short_key_range(cuda_lib, M, L, H):
+    """Key ranges of at most 8 tiles (the cross-attention's context) run the persistent
+    one-parity kernel, two CTAs per SM, each walking its units: exact query tiles, ragged last
+    query tiles (300, 200, 2000, 129, 100, 40000, 20000 rows), a single query row, a single ragged
+    key tile (16 keys), the largest range that takes this path (1024 keys), a ragged 129-key
+    range, and more units than CTAs (313 and 471 units: some CTAs take two, across heads)."""
     D = 128 * H
     q = S.normal(91, (M, D), 2.0, True)
     k, v = S.normal(92, (L, D), 1.0, True), S.normal(93, (L, D), 1.0, True)
@@ -246,12 +253,12 @@ def test_attention_two_query_tiles(cuda_lib, M, L, H):
     o = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
     cuda_lib.attention(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), H, o)
     assert cuda_lib.device_status() == 0
-    assert_bf16_close(host(o), O.attention(q, k, v), "attention, two query tiles per CTA")
+    assert_bf16_close(host(o), O.attention(q, k, v), "attention, short key range")
 
 
-def test_attention_two_query_tiles_wan_cross(cuda_lib):
+def test_attention_short_key_range_wan_cross(cuda_lib):
     """The Wan-1.3B cross-attention shape: 32760 queries against the 512-row context, 12 heads
-    (64 pairs of query tiles per head, the last one ragged); sampled rows against the oracle."""
+    (256 query tiles per head, the last one ragged); sampled rows against the oracle."""
     M, L, H = 32760, 512, 12
     D = 128 * H
     q = S.normal(94, (M, D), 1.0, True)

@@ -33,13 +33,13 @@ static int launch_ln(float* X, const float* x_src, const int* idx, int M, int N,
   ScopedTiming timing(HSA_KCLASS_OTHER, st);
   const unsigned g = warp_blocks(M);
   switch (D / 128 * (D % 128 == 0)) {
-    case 1: k_ln_rows<1, TOut><<<g, 256, 0, st>>>(X, x_src, idx, M, N, mul, add, plus_one, h); break;
-    case 2: k_ln_rows<2, TOut><<<g, 256, 0, st>>>(X, x_src, idx, M, N, mul, add, plus_one, h); break;
-    case 4: k_ln_rows<4, TOut><<<g, 256, 0, st>>>(X, x_src, idx, M, N, mul, add, plus_one, h); break;
-    case 8: k_ln_rows<8, TOut><<<g, 256, 0, st>>>(X, x_src, idx, M, N, mul, add, plus_one, h); break;
-    case 12: k_ln_rows<12, TOut><<<g, 256, 0, st>>>(X, x_src, idx, M, N, mul, add, plus_one, h); break;
-    case 16: k_ln_rows<16, TOut><<<g, 256, 0, st>>>(X, x_src, idx, M, N, mul, add, plus_one, h); break;
-    default: k_ln_rows_any<TOut><<<g, 256, 0, st>>>(X, x_src, idx, M, N, D, mul, add, plus_one, h); break;
+    case 1: launch(k_ln_rows<1, TOut>, g, 256, 0, st, X, x_src, idx, M, N, mul, add, plus_one, h); break;
+    case 2: launch(k_ln_rows<2, TOut>, g, 256, 0, st, X, x_src, idx, M, N, mul, add, plus_one, h); break;
+    case 4: launch(k_ln_rows<4, TOut>, g, 256, 0, st, X, x_src, idx, M, N, mul, add, plus_one, h); break;
+    case 8: launch(k_ln_rows<8, TOut>, g, 256, 0, st, X, x_src, idx, M, N, mul, add, plus_one, h); break;
+    case 12: launch(k_ln_rows<12, TOut>, g, 256, 0, st, X, x_src, idx, M, N, mul, add, plus_one, h); break;
+    case 16: launch(k_ln_rows<16, TOut>, g, 256, 0, st, X, x_src, idx, M, N, mul, add, plus_one, h); break;
+    default: launch(k_ln_rows_any<TOut>, g, 256, 0, st, X, x_src, idx, M, N, D, mul, add, plus_one, h); break;
   }
   count_launch(1);
   return check_launch("layernorm launch");
@@ -51,12 +51,12 @@ static int launch_qk_rope(const T* qkv, const int* idx, const int* pos, int M, i
   ScopedTiming timing(HSA_KCLASS_OTHER, st);
   const unsigned g = warp_blocks(M);
   switch (D / 128) {
-    case 1: k_qk_norm_rope<1, T, T><<<g, 256, 0, st>>>(qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
-    case 2: k_qk_norm_rope<2, T, T><<<g, 256, 0, st>>>(qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
-    case 4: k_qk_norm_rope<4, T, T><<<g, 256, 0, st>>>(qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
-    case 8: k_qk_norm_rope<8, T, T><<<g, 256, 0, st>>>(qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
-    case 12: k_qk_norm_rope<12, T, T><<<g, 256, 0, st>>>(qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
-    default: k_qk_norm_rope_any<T, T><<<g, 256, 0, st>>>(qkv, idx, pos, M, N, D, g_q, g_k, Q, Kc, Vc); break;
+    case 1: launch(k_qk_norm_rope<1, T, T>, g, 256, 0, st, qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
+    case 2: launch(k_qk_norm_rope<2, T, T>, g, 256, 0, st, qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
+    case 4: launch(k_qk_norm_rope<4, T, T>, g, 256, 0, st, qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
+    case 8: launch(k_qk_norm_rope<8, T, T>, g, 256, 0, st, qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
+    case 12: launch(k_qk_norm_rope<12, T, T>, g, 256, 0, st, qkv, idx, pos, M, N, g_q, g_k, Q, Kc, Vc); break;
+    default: launch(k_qk_norm_rope_any<T, T>, g, 256, 0, st, qkv, idx, pos, M, N, D, g_q, g_k, Q, Kc, Vc); break;
   }
   count_launch(1);
   return check_launch("qk norm / rope launch");
@@ -66,7 +66,7 @@ template <typename T>
 static int launch_rms(const T* in, int in_stride, int M, int D, const float* g, T* out, cudaStream_t st) {
   if (M <= 0) return HSA_OK;
   ScopedTiming timing(HSA_KCLASS_OTHER, st);
-  k_rms_rows<T, T><<<warp_blocks(M), 256, 0, st>>>(in, in_stride, M, D, g, out);
+  launch(k_rms_rows<T, T>, warp_blocks(M), 256, 0, st, in, in_stride, M, D, g, out);
   count_launch(1);
   return check_launch("rms rows launch");
 }
@@ -99,7 +99,7 @@ extern "C" int hsa_l1_score(const float* d_v_new, const float* d_v_prev, int N, 
   if (!d_v_new || !d_v_prev || !d_score || !aligned16(d_v_new) || !aligned16(d_v_prev))
     return set_error(HSA_EINVAL, "l1_score: null or misaligned pointer");
   ScopedTiming timing(HSA_KCLASS_OTHER, as_stream(stream));
-  k_l1_score<<<warp_blocks(N), 256, 0, as_stream(stream)>>>(d_v_new, d_v_prev, N, C, d_score);
+  launch(k_l1_score, warp_blocks(N), 256, 0, as_stream(stream), d_v_new, d_v_prev, N, C, d_score);
   count_launch(1);
   return check_launch("l1_score launch");
 }
@@ -115,19 +115,21 @@ extern "C" int hsa_euler_update(float* d_x, float* d_vhat, const float* d_vA, co
   ScopedTiming timing(HSA_KCLASS_OTHER, st);
   if (M == N) {
     // every token active: scatter, score and Euler in one pass over the rows
-    k_scatter_vhat<<<warp_blocks(M), 256, 0, st>>>(d_vhat, d_vA, d_idx, M, N, C, d_score, d_x, dsigma);
+    launch(k_scatter_vhat, warp_blocks(M), 256, 0, st, d_vhat, d_vA, d_idx, M, N, C, d_score, d_x, dsigma);
     count_launch(1);
     return check_launch("euler (full step) launch");
   }
   if (M > 0) {
-    k_scatter_vhat<<<warp_blocks(M), 256, 0, st>>>(d_vhat, d_vA, d_idx, M, N, C, d_score, nullptr, dsigma);
+    launch(k_scatter_vhat, warp_blocks(M), 256, 0, st, d_vhat, d_vA, d_idx, M, N, C, d_score, nullptr, dsigma);
     count_launch(1);
     HSA_TRY(check_launch("v_hat scatter launch"));
   }
   const size_t n4 = (size_t)N * C / 4;
-  const size_t want = (n4 + 1023) / 1024;   // 4 float4 per thread per iteration
-  const size_t cap = (size_t)num_sms() * 8;
-  k_euler<<<(unsigned)(want < cap ? want : cap), 256, 0, st>>>(d_x, d_vhat, n4, dsigma);
+  // up to 4 float4 per thread per pass; the same number of 256-thread blocks on every SM (at most
+  // 8, a full SM), so no SM holds one block more than another
+  const size_t sms = (size_t)num_sms();
+  const size_t per_sm = ((n4 + 1023) / 1024 + sms - 1) / sms;
+  launch(k_euler, (unsigned)(sms * (per_sm < 8 ? per_sm : 8)), 256, 0, st, d_x, d_vhat, n4, dsigma);
   count_launch(1);
   return check_launch("euler launch");
 }
@@ -307,9 +309,10 @@ extern "C" int hsa_patch_embed(const float* d_x, const int32_t* d_idx, int M, in
   cudaStream_t st = as_stream(stream);
   ScopedTiming timing(HSA_KCLASS_OTHER, st);
   if (dtype == HSA_BF16)
-    k_gather_rows<__nv_bfloat16><<<warp_blocks(M), 256, 0, st>>>(d_x, d_idx, M, N, C, static_cast<__nv_bfloat16*>(d_ws));
+    launch(k_gather_rows<__nv_bfloat16>, warp_blocks(M), 256, 0, st, d_x, d_idx, M, N, C,
+           static_cast<__nv_bfloat16*>(d_ws));
   else
-    k_gather_rows<float><<<warp_blocks(M), 256, 0, st>>>(d_x, d_idx, M, N, C, static_cast<float*>(d_ws));
+    launch(k_gather_rows<float>, warp_blocks(M), 256, 0, st, d_x, d_idx, M, N, C, static_cast<float*>(d_ws));
   count_launch(1);
   HSA_TRY(check_launch("gather launch"));
   return linear(d_ws, M, C, d_w_in, D, d_b_in, dtype, HSA_EPI_F32, nullptr, d_X, st);

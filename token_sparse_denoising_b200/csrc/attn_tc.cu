@@ -6,7 +6,9 @@
 //   o = softmax(q K^T / sqrt(128)) V, per head; q: M x 128H compacted rows,
 //   K, V: L x 128H cache rows, o: M x 128H.  Non-causal.
 //
-// One CTA = one head x 128 queries, streaming 128-key tiles of K and V.
+// One CTA = one head x 128 queries, streaming 128-key tiles of K and V.  Two variants share the
+// code: k_attn_tc<2> (two tile parities, one CTA per SM) for long key ranges, k_attn_tc<1> (one
+// parity, two CTAs per SM) for short ones.  k_attn_tc<2>:
 //   warp 0      TMA producer (the warp waits, one elected lane copies): Q once; K_j into a
 //               3-slot ring, V_j into a 2-slot ring, in the order the MMA warp consumes
 //               them (K0 K1 V0 K2 V1 K3 ...).  V_j and K_{j+2} complete on the barriers
@@ -35,6 +37,17 @@
 // first 64 columns of S_b.  QK^T of tile j+2 overwrites S_b only after PV of tile j
 // has read P_b: both are issued by the one MMA thread, whose tcgen05.mma operations
 // execute in issue order.
+// k_attn_tc<1> runs the same steps with one parity: warps 2..5 take every tile, TMEM holds S
+// [0,128) and O [128,256), K and V have one slot each, and QK^T of tile j+1 follows PV of tile
+// j.  A CTA's chain of tiles is then serial, but it needs half the shared memory, TMEM and
+// threads, so two CTAs share an SM and one's tiles overlap the other's.  The CTAs are persistent:
+// each walks units blockIdx.x, blockIdx.x + gridDim.x, ..., with Q of the next unit loaded once
+// the last QK^T of the current one is done, and the K of the next unit's first tile bundled with
+// the current unit's last P, so the next unit's first QK^T follows the last PV at once.  The
+// epilogue stages O in the V slot (the next unit's first V waits for it) and releases O to the
+// next unit's first PV as soon as it is in registers.  With a few key tiles per unit (the
+// cross-attention's 512-row context) CTA set-up, Q latency and the epilogue were most of a
+// unit's time when every unit was a CTA of its own.
 // Key rows beyond L are zero-filled by TMA and masked to -inf; query rows beyond
 // M are computed on zeros and never stored.
 //
@@ -49,13 +62,11 @@ namespace hsa {
 
 constexpr int kAttnBM = 128;
 constexpr int kAttnBN = 128;
-constexpr int kKSlots = 3;
-// Key ranges of at most this many 128-key tiles run two query tiles per CTA (k_attn_tc<true>)
-constexpr int kTwoQMaxTiles = 8;
-constexpr int kVSlots = 2;
-constexpr int kAttnThreads = 320;                 // 2 control warps + 8 softmax warps
+// Key ranges of at most this many 128-key tiles run the one-parity kernel (k_attn_tc<1>), two
+// CTAs per SM; longer ones the two-parity kernel (k_attn_tc<2>), one CTA per SM
+constexpr int kShortMaxTiles = 8;
 constexpr int kTileBytes = 128 * 128 * 2;         // one 128 x 128 bf16 operand tile (two 64-column boxes)
-constexpr uint32_t kColS = 0, kColO = 256;
+constexpr uint32_t kColS = 0;
 // Exponentials computed with the polynomial instead of the MUFU unit: the columns c
 // of a thread's 128 with (c % 8) >= 8 - kPolyPer8.  Every measurement at the Wan-1.3B
 // shape (attention alone, 32760 x 32760, 12 heads) found the MUFU path faster: with two
@@ -65,22 +76,42 @@ constexpr uint32_t kColS = 0, kColO = 256;
 #define HSA_ATTN_POLY_PER8 0
 #endif
 constexpr int kPolyPer8 = HSA_ATTN_POLY_PER8;
+#ifndef HSA_ATTN_POLY_SHORT_PER8
+#define HSA_ATTN_POLY_SHORT_PER8 0
+#endif
 // P goes to the MMA warp in two halves of 64 keys; PV of the first half starts while the
 // softmax warps compute the exponentials of the second.  Measured at the Wan-1.3B shape
 // (attention alone): one release per tile 5.40 ms, halves 5.21 ms, quarters 5.47 ms.
 
 struct AttnShared {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[kKSlots];    // k_full: tiles 0 and 1 only
-  uint64_t v_empty[kVSlots];
-  // p_full[b][h]: P of keys [64 h, 64 h + 64) of tile j (b = j % 2) stored by the 128 softmax
-  // threads, plus one producer arrival with the bytes of the next operand the MMA warp needs:
-  // V_j for h = 0, K_{j+2} for h = 1 (a plain arrival when there is no tile j+2)
+  uint64_t k_full[2], k_empty[3];    // k_full: the first tile of each parity only
+  uint64_t v_empty[2];
+  // p_full[b][h]: P of keys [64 h, 64 h + 64) of tile t (b = t % kPar) stored by the 128 softmax
+  // threads of parity b, plus one producer arrival with the bytes of the next operand the MMA
+  // warp needs: V_t for h = 0, K_{t+kPar} for h = 1 (a plain arrival when there is no such tile)
   uint64_t s_full[2], p_full[2][2], o_done;
+  // one-parity kernel, which walks several units: Q reusable (last QK^T of a unit done), O read
+  // out by the epilogue, staging area (the V slot) read back by the epilogue
+  uint64_t q_empty, o_free, stage_free;
   uint32_t tmem;
   float xm[2][128], xl[2][128];  // [parity][row]: running max and sum, merged in the epilogue
 };
-constexpr int kAttnSmem = kTileBytes * (1 + kKSlots + kVSlots) + 1024 + (int)sizeof(AttnShared);
+
+// The two variants.  kPar = 2: 2 control warps + 8 softmax warps, TMEM S0 S1 O0 O1 (512
+// columns), a 3-slot K ring and a 2-slot V ring, one CTA per SM.  kPar = 1: 2 control warps + 4
+// softmax warps, TMEM S O (256 columns), one K and one V slot, two CTAs per SM, so one CTA's
+// fill and drain overlap the other's tiles.
+template <int kPar>
+struct AttnCfg {
+  static constexpr int kThreads = 64 + 128 * kPar;
+  static constexpr int kKSlots = kPar == 2 ? 3 : 1;
+  static constexpr int kVSlots = kPar == 2 ? 2 : 1;
+  static constexpr uint32_t kCols = 256 * kPar;
+  static constexpr uint32_t kColO = 128 * kPar;
+  static constexpr int kSmem = kTileBytes * (1 + kKSlots + kVSlots) + 1024 + (int)sizeof(AttnShared);
+};
+static_assert(2 * AttnCfg<1>::kSmem <= 227 * 1024, "two one-parity CTAs must fit one SM's shared memory");
 
 // Unit -> CTA map: units u < u_full are whole; unit u_full + t / s_tail, key range t % s_tail,
 // for the split tail.  part_o / part_ml hold the split CTAs' partial results, slot t.
@@ -142,32 +173,25 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// kTwoQ: the CTA takes two 128-query tiles of one head (256 queries) and streams each key tile
-// once for both.  Virtual tile t = 2 j + b is key tile j of query tile b, so the parity of a
-// virtual tile is its query tile, and the parity machinery below (S, O and softmax warps per
-// parity, the MMA issue order) runs over 2 nj virtual tiles.  K_j and V_j are loaded once, with
-// the even virtual tile's barriers, and released after the odd virtual tile's QK^T / PV; the
-// parity-1 P barriers count the softmax threads alone (the producer has nothing to add there),
-// and the producer waits for the previous phase of the parity-0 barriers before arriving on them
-// (its ring slots come back only two phases after their last use, which alone would let an
-// arrival land in the phase before its own); the epilogue writes each parity's own rows instead
-// of merging the two.  Used for short key ranges (the cross-attention's
-// context), where filling and draining the pipeline dominates a unit.
-template <bool kTwoQ>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+template <int kPar>
+__global__ void __launch_bounds__(AttnCfg<kPar>::kThreads, 3 - kPar)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, int M, int L, int H, __nv_bfloat16* __restrict__ O,
               const AttnGrid grid) {
+  pdl_prologue();
+  using Cfg = AttnCfg<kPar>;
+  constexpr int KS = Cfg::kKSlots, VS = Cfg::kVSlots;
+  constexpr uint32_t kColO = Cfg::kColO;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  constexpr int QTILES = kTwoQ ? 2 : 1;                 // query tiles of the CTA
-  constexpr int KS = kTwoQ ? 2 : kKSlots;                // K ring slots (shared memory: 6 tiles either way)
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + QTILES * kTileBytes;              // slot s at s * kTileBytes
+  uint8_t* sK = smem + kTileBytes;                       // slot s at s * kTileBytes
   uint8_t* sV = sK + KS * kTileBytes;
-  AttnShared* sh = reinterpret_cast<AttnShared*>(sV + kVSlots * kTileBytes);
+  AttnShared* sh = reinterpret_cast<AttnShared*>(sV + VS * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // kPar == 1 walks units blockIdx.x, blockIdx.x + gridDim.x, ... (all whole); kPar == 2 takes one
+  const int n_units = kPar == 1 ? (grid.u_full - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 1;
   int u = blockIdx.x, split = 0, n_split = 1, slot = -1;
   if (u >= grid.u_full) {
     const int t = u - grid.u_full;
@@ -176,36 +200,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     n_split = grid.s_tail;
     if (n_split > 1) slot = t;
   }
-  const int m0 = (u % grid.QT) * kAttnBM * QTILES, h = u / grid.QT;
-  // this CTA's key tiles [j0, j0 + nj): loops, ring slots and parities use the local index
+  const int m0 = (u % grid.QT) * kAttnBM, h = u / grid.QT;
+  // this CTA's key tiles [j0, j0 + nt): loops, ring slots and parities use the local index
   const int nj_all = (L + kAttnBN - 1) / kAttnBN;
   const int j0 = split * nj_all / n_split;
-  const int nj = (split + 1) * nj_all / n_split - j0;
-  const int nt = kTwoQ ? 2 * nj : nj;                    // virtual tiles (key tile x query tile)
-  // key tile of virtual tile t
-  auto key_of = [](int t) { return kTwoQ ? t >> 1 : t; };
+  const int nt = (split + 1) * nj_all / n_split - j0;
 
   if (threadIdx.x == 0) {
     mbar_init(&sh->q_full, 1);
     for (int s = 0; s < KS; ++s) mbar_init(&sh->k_empty[s], 1);
-    for (int s = 0; s < 2; ++s) mbar_init(&sh->k_full[s], 1);
-    for (int s = 0; s < kVSlots; ++s) mbar_init(&sh->v_empty[s], 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kPar; ++b) mbar_init(&sh->k_full[b], 1);
+    for (int s = 0; s < VS; ++s) mbar_init(&sh->v_empty[s], 1);
+    for (int b = 0; b < kPar; ++b) {
       mbar_init(&sh->s_full[b], 1);
-      // the softmax threads, plus one producer arrival (with the bytes of V_j / the next K) where
-      // the producer has something to deliver: every tile, or the even virtual tiles of kTwoQ
-      const uint32_t n_arrive = (kTwoQ && b == 1) ? 128 : 129;
-      mbar_init(&sh->p_full[b][0], n_arrive);
-      mbar_init(&sh->p_full[b][1], n_arrive);
+      mbar_init(&sh->p_full[b][0], 129);   // the parity's 128 softmax threads + the producer
+      mbar_init(&sh->p_full[b][1], 129);
     }
     mbar_init(&sh->o_done, 1);
+    if (kPar == 1) {
+      mbar_init(&sh->q_empty, 1);
+      mbar_init(&sh->o_free, 128);
+      mbar_init(&sh->stage_free, 128);
+    }
     fence_mbar_init();
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
   }
   if (warp == 1) {
-    tmem_alloc(&sh->tmem, 512);
+    tmem_alloc(&sh->tmem, Cfg::kCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -213,19 +236,72 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tm = sh->tmem;
 
-  if (warp == 0) {
+  if (warp == 0 && kPar == 1) {
+    // TMA producer of the one-parity kernel, unit after unit (T counts this CTA's tiles over all
+    // of its units): Q of unit i once the last QK^T of unit i-1 is done, so it arrives while
+    // that unit finishes; K and V of every tile in order, the K of tile T + 1 (the next unit's
+    // first at a unit's end) completing with the second half of P_T.  The V slot doubles as the
+    // epilogue's staging area, so the first V of a unit also waits until the previous unit's
+    // output has been read back out of it.
+    const bool leader = elect_one();
+    const int ntot = n_units * nt;
+    auto unit_of = [&](int i) { return (int)blockIdx.x + i * (int)gridDim.x; };
+    auto load_k = [&](int T, uint64_t* bar) -> bool {
+      const bool ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->k_empty[0], (T & 1) ^ 1), 0);
+      __syncwarp();
+      if (ok && leader) {
+        const int x0 = unit_of(T / nt) / grid.QT * 128, row = (T % nt) * kAttnBN;
+        mbar_expect_tx(bar, kTileBytes);
+        tma_load_2d(sK, &tmK, bar, x0, row);
+        tma_load_2d(sK + kTileBytes / 2, &tmK, bar, x0 + 64, row);
+      }
+      return ok;
+    };
+    bool ok = true;
+    for (int i = 0; ok && i < n_units; ++i) {
+      const int ui = unit_of(i), x0 = ui / grid.QT * 128;
+      if (i > 0) {
+        ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->q_empty, (i - 1) & 1), 0);
+        __syncwarp();
+        if (!ok) break;
+      }
+      if (leader) {
+        const int row = ui % grid.QT * kAttnBM;
+        mbar_expect_tx(&sh->q_full, kTileBytes);
+        tma_load_2d(sQ, &tmQ, &sh->q_full, x0, row);
+        tma_load_2d(sQ + kTileBytes / 2, &tmQ, &sh->q_full, x0 + 64, row);
+      }
+      __syncwarp();
+      if (i == 0) ok = load_k(0, &sh->k_full[0]);
+      for (int t = 0; ok && t < nt; ++t) {
+        const int T = i * nt + t;
+        ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->v_empty[0], (T & 1) ^ 1), 0);
+        if (ok && t == 0 && i > 0) ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->stage_free, (i - 1) & 1), 0);
+        __syncwarp();
+        if (!ok) break;
+        if (leader) {
+          mbar_expect_tx(&sh->p_full[0][0], kTileBytes);
+          tma_load_2d(sV, &tmV, &sh->p_full[0][0], x0, t * kAttnBN);
+          tma_load_2d(sV + kTileBytes / 2, &tmV, &sh->p_full[0][0], x0 + 64, t * kAttnBN);
+        }
+        if (T + 1 < ntot) {
+          ok = load_k(T + 1, &sh->p_full[0][1]);
+        } else {
+          if (leader) mbar_arrive(&sh->p_full[0][1]);
+          __syncwarp();
+        }
+      }
+    }
+  } else if (warp == 0) {
     // TMA producer: the whole warp runs the loop and waits; one elected lane issues the copies
     const int x0 = h * 128;
     const bool leader = elect_one();
     if (leader) {
-      mbar_expect_tx(&sh->q_full, QTILES * kTileBytes);
-#pragma unroll
-      for (int qt = 0; qt < QTILES; ++qt) {
-        tma_load_2d(sQ + qt * kTileBytes, &tmQ, &sh->q_full, x0, m0 + qt * kAttnBM);
-        tma_load_2d(sQ + qt * kTileBytes + kTileBytes / 2, &tmQ, &sh->q_full, x0 + 64, m0 + qt * kAttnBM);
-      }
+      mbar_expect_tx(&sh->q_full, kTileBytes);
+      tma_load_2d(sQ, &tmQ, &sh->q_full, x0, m0);
+      tma_load_2d(sQ + kTileBytes / 2, &tmQ, &sh->q_full, x0 + 64, m0);
     }
-    // K of key tile j into its ring slot, completing on `bar`
+    // K of tile j into its ring slot, completing on `bar`
     auto load_k = [&](int j, uint64_t* bar) -> bool {
       const int sk = j % KS;
       const bool ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->k_empty[sk], ((j / KS) & 1) ^ 1), 0);
@@ -239,35 +315,84 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       return ok;
     };
     bool ok = load_k(0, &sh->k_full[0]);
-    if (!kTwoQ && ok && nj > 1) ok = load_k(1, &sh->k_full[1]);
-    static_assert(kVSlots == 2, "V slot j % 2 is also the parity of tile j");
-    // kTwoQ: only the even virtual tiles (t = 2 j) have something to deliver -- V_j, and the K of
-    // QK^T(t + 2) = K_{j+1}; the odd ones read the same V_j and issue QK^T with K_{j+1} after the
-    // even tile's barriers completed, so the producer skips them
-    for (int t = 0; ok && t < nt; t += kTwoQ ? 2 : 1) {
-      const int b = t & 1, j = key_of(t), sv = j & 1;
-      ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->v_empty[sv], ((j >> 1) & 1) ^ 1), 0);
+    if (kPar == 2 && ok && nt > 1) ok = load_k(1, &sh->k_full[1]);
+    // Phase order of the p_full arrivals: the producer arrives on phase (t / kPar) of
+    // p_full[t % kPar][*] only after waiting for a ring slot that the MMA warp releases after it
+    // waited on the previous phase of the same barrier, so no arrival lands a phase early
+    for (int t = 0; ok && t < nt; ++t) {
+      const int b = t % kPar, sv = t % VS;
+      ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->v_empty[sv], ((t / VS) & 1) ^ 1), 0);
       __syncwarp();
-      if (kTwoQ && ok && j > 0) {
-        // a ring slot comes back two phases after its last use here, so wait for the previous
-        // phase of both barriers before arriving on them: an arrival is never counted early
-        ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->p_full[0][0], (j - 1) & 1), 0);
-        if (ok) ok = __shfl_sync(0xffffffffu, mbar_wait(&sh->p_full[0][1], (j - 1) & 1), 0);
-        __syncwarp();
-      }
       if (!ok) break;
       if (leader) {
         uint8_t* v = sV + sv * kTileBytes;
         mbar_expect_tx(&sh->p_full[b][0], kTileBytes);
-        tma_load_2d(v, &tmV, &sh->p_full[b][0], x0, (j0 + j) * kAttnBN);
-        tma_load_2d(v + kTileBytes / 2, &tmV, &sh->p_full[b][0], x0 + 64, (j0 + j) * kAttnBN);
+        tma_load_2d(v, &tmV, &sh->p_full[b][0], x0, (j0 + t) * kAttnBN);
+        tma_load_2d(v + kTileBytes / 2, &tmV, &sh->p_full[b][0], x0 + 64, (j0 + t) * kAttnBN);
       }
-      if (t + 2 < nt) {
-        ok = load_k(key_of(t + 2), &sh->p_full[b][1]);
+      if (t + kPar < nt) {
+        ok = load_k(t + kPar, &sh->p_full[b][1]);
       } else {
         if (leader) mbar_arrive(&sh->p_full[b][1]);
         __syncwarp();
       }
+    }
+  } else if (warp == 1 && kPar == 1) {
+    // MMA issuer of the one-parity kernel, unit after unit: S = Q K_T^T, then P_T V_T in two
+    // halves into O, then the next QK^T.  A unit's first PV overwrites O, so it waits until the
+    // epilogue has read the previous unit's O out of TMEM; the unit's last QK^T frees Q.
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
+    const bool leader = elect_one();
+    const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t k_desc = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t v_desc = sdesc_sw128(smem_u32(sV), kTileBytes / 2, 1024);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      const bool r = __shfl_sync(0xffffffffu, mbar_wait(bar, parity), 0);
+      __syncwarp();
+      return r;
+    };
+    // QK^T of the tile whose K is in the slot; `last`: the unit's last, after which Q is free
+    auto issue_qk = [&](bool last) {
+      tc_fence_after();
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
+          umma_ss(tm + kColS, q_desc + off, k_desc + off, idesc_s, kk > 0);
+        }
+        umma_commit(&sh->s_full[0]);
+        umma_commit(&sh->k_empty[0]);
+        if (last) umma_commit(&sh->q_empty);
+      }
+      __syncwarp();
+    };
+    bool ok = true;
+    for (int i = 0; ok && i < n_units; ++i) {
+      ok = wait_all(&sh->q_full, i & 1);
+      if (ok && i == 0) ok = wait_all(&sh->k_full[0], 0);
+      if (!ok) break;
+      issue_qk(nt == 1);
+      for (int t = 0; ok && t < nt; ++t) {
+        const int T = i * nt + t;
+        if (t == 0 && i > 0 && !wait_all(&sh->o_free, (i - 1) & 1)) { ok = false; break; }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          // half 0 also brings V_T, half 1 also the K of the next tile
+          if (!wait_all(&sh->p_full[0][q], T & 1)) { ok = false; break; }
+          tc_fence_after();
+          if (leader) {
+#pragma unroll
+            for (int kk = q * 4; kk < q * 4 + 4; ++kk)
+              umma_ts(tm + kColO, tm + kColS + kk * 8, v_desc + (uint64_t)(kk * 2048 >> 4), idesc_o, (t > 0 || kk > 0));
+            if (q == 1) umma_commit(&sh->v_empty[0]);
+          }
+          __syncwarp();
+        }
+        if (ok && t + 1 < nt) issue_qk(t + 2 == nt);   // overwrites S (P_T) after PV_T in issue order
+      }
+      if (leader) umma_commit(&sh->o_done);   // every MMA of the unit
+      __syncwarp();
     }
   } else if (warp == 1) {
     // MMA issuer: the whole warp runs the loop, waits and builds the descriptors (warp-uniform
@@ -285,31 +410,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       return r;
     };
-    // QK^T of virtual tile t; the first two wait for their K here, later ones through p_full
+    // QK^T of tile t; the first tile of each parity waits for its K here, later ones through p_full
     auto issue_qk = [&](int t) -> bool {
-      const int j = key_of(t), sk = j % KS, b = t & 1;
-      if (t < 2 && !wait_all(&sh->k_full[kTwoQ ? 0 : t], 0)) return false;
+      const int sk = t % KS, b = t % kPar;
+      if (t < kPar && !wait_all(&sh->k_full[t], 0)) return false;
       tc_fence_after();
       const uint64_t kd = k_desc + (uint64_t)((sk * kTileBytes) >> 4);
-      const uint64_t qd = q_desc + (uint64_t)(((kTwoQ ? b : 0) * kTileBytes) >> 4);
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
-          umma_ss(tm + kColS + b * 128, qd + off, kd + off, idesc_s, kk > 0);
+          umma_ss(tm + kColS + b * 128, q_desc + off, kd + off, idesc_s, kk > 0);
         }
         umma_commit(&sh->s_full[b]);
-        // K_j is free once every S it feeds is computed
-        if (!kTwoQ || b == 1) umma_commit(&sh->k_empty[sk]);
+        umma_commit(&sh->k_empty[sk]);   // K_t is free once S_t is computed
       }
       __syncwarp();
       return true;
     };
     bool ok = wait_all(&sh->q_full, 0);
     if (ok) ok = issue_qk(0);
-    if (ok && nt > 1) ok = issue_qk(1);
+    if (kPar == 2 && ok && nt > 1) ok = issue_qk(1);
     for (int t = 0; ok && t < nt; ++t) {
-      const int b = t & 1, j = key_of(t), sv = j % kVSlots;
+      const int b = t % kPar, sv = t % VS;
       const uint64_t vd = v_desc + (uint64_t)((sv * kTileBytes) >> 4);
 
       // PV half by half of the keys: the first starts while the softmax warps are still
@@ -317,25 +440,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool got = true;
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        // half 0 also brings V_j, half 1 also the K of QK^T(t + 2) (even virtual tiles only with kTwoQ)
-        if (!wait_all(&sh->p_full[b][q], (t >> 1) & 1)) { got = false; break; }
+        // half 0 also brings V_t, half 1 also the K of QK^T(t + kPar)
+        if (!wait_all(&sh->p_full[b][q], (t / kPar) & 1)) { got = false; break; }
         tc_fence_after();
         if (leader) {
 #pragma unroll
           for (int kk = q * 4; kk < q * 4 + 4; ++kk) {
             // V tile: key rows of 128 B (64 channels) per box; 16 keys = two 1024-byte atoms
             umma_ts(tm + kColO + b * 128, tm + kColS + b * 128 + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), idesc_o,
-                    (t >= 2 || kk > 0));
+                    (t >= kPar || kk > 0));
           }
-          // V_j is free once every PV that reads it is issued
-          if (q == 1 && (!kTwoQ || b == 1)) umma_commit(&sh->v_empty[sv]);
+          if (q == 1) umma_commit(&sh->v_empty[sv]);   // V_t is free once PV_t is done
         }
         __syncwarp();
       }
       if (!got) break;
-      if (t + 2 < nt) ok = issue_qk(t + 2);   // overwrites S_b (P_t) after PV_t in issue order
+      if (t + kPar < nt) ok = issue_qk(t + kPar);   // overwrites S_b (P_t) after PV_t in issue order
     }
-    if (leader) umma_commit(&sh->o_done);   // every MMA of this CTA, both O accumulators
+    if (leader) umma_commit(&sh->o_done);   // every MMA of this CTA
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax warps
@@ -345,10 +467,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_base = tm + ((uint32_t)(quarter * 32) << 16);
     const uint32_t s_col = lane_base + kColS + par * 128, o_col = lane_base + kColO + par * 128;
     const float sc = 0.12751743074680484f;          // log2(e) / sqrt(128)
+    for (int iu = 0; iu < n_units; ++iu) {   // one unit unless kPar == 1
     float m = -INFINITY, l = 0.f;
-    for (int t = par; t < nt; t += 2) {
-      const int j = key_of(t);
-      mbar_wait(&sh->s_full[par], (t >> 1) & 1);
+    for (int t = par; t < nt; t += kPar) {
+      mbar_wait(&sh->s_full[par], ((iu * nt + t) / kPar) & 1);
       __syncwarp();
       tc_fence_after();
       uint32_t sr[128];
@@ -357,8 +479,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld32(s_col + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + q4 * 32));
       tmem_ld_wait();
 
-      if ((j0 + j + 1) * kAttnBN > L) {  // ragged last tile only: keys beyond L get -inf
-        const int valid = L - (j0 + j) * kAttnBN;
+      if ((j0 + t + 1) * kAttnBN > L) {  // ragged last tile only: keys beyond L get -inf
+        const int valid = L - (j0 + t) * kAttnBN;
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
@@ -395,7 +517,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int c = hh * 64; c < hh * 64 + 64; c += 2) {
           const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
-          const bool poly = (c & 7) >= 8 - kPolyPer8;  // compile-time per unrolled column pair
+          // compile-time per unrolled column pair
+          const bool poly = (c & 7) >= 8 - (kPar == 1 ? HSA_ATTN_POLY_SHORT_PER8 : kPolyPer8);
           const float p0 = poly ? ex2_poly(x.x) : ex2_approx(x.x);
           const float p1 = poly ? ex2_poly(x.y) : ex2_approx(x.y);
           rs4[(c >> 1) & 3] = fadd2(rs4[(c >> 1) & 3], make_float2(p0, p1));
@@ -432,38 +555,56 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(&sh->p_full[par][1]);
     }
     // ---------------------------------------------------------------- epilogue
-    if constexpr (kTwoQ) {
-      // each parity holds its own query tile: O_par / l for rows m0 + 128 par + row
-      mbar_wait(&sh->o_done, 0);
+    if constexpr (kPar == 1) {
+      // one parity, whole key range (the host never splits these units): O / l of unit iu
+      mbar_wait(&sh->o_done, iu & 1);
       __syncwarp();
       tc_fence_after();
-      const int grow = m0 + par * kAttnBM + row;
+      const int ui = (int)blockIdx.x + iu * (int)gridDim.x;
+      const int m0u = ui % grid.QT * kAttnBM, hu = ui / grid.QT;
       const float inv_l = 1.0f / l;
+      // The unit's last PV is done, so the V slot is free until this warp's stage_free arrival:
+      // the warp stages its 32 rows there (256 B each, the 16-byte chunks of row r XOR-rotated by
+      // r % 16), then writes them out with 16 lanes per row, two whole rows per store instead of
+      // 32 rows' fragments.  O is released to the next unit's first PV once it is in registers.
+      uint8_t* stage = sV + quarter * (32 * 256);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         __syncwarp();
         tmem_ld32(o_col + c * 32, o);
         tmem_ld_wait();
-        if (grow < M) {
-          __nv_bfloat16* dst = O + (size_t)grow * (H * 128) + h * 128 + c * 32;
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 pk4;
-            pk4.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
-            pk4.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
-            pk4.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
-            pk4.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
-            *reinterpret_cast<uint4*>(dst + e) = pk4;
-          }
+        for (int e = 0; e < 32; e += 8) {
+          uint4 pk4;
+          pk4.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+          pk4.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+          pk4.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+          pk4.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+          const int chunk = c * 4 + (e >> 3);
+          *reinterpret_cast<uint4*>(stage + lane * 256 + ((chunk ^ (lane & 15)) << 4)) = pk4;
         }
       }
+      tc_fence_before();
+      mbar_arrive(&sh->o_free);
+      __syncwarp();
+      const int cl = lane & 15;
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        const int r = 2 * i + (lane >> 4);
+        const uint4 val = *reinterpret_cast<const uint4*>(stage + r * 256 + ((cl ^ (r & 15)) << 4));
+        const int grow = m0u + quarter * 32 + r;
+        if (grow < M) *reinterpret_cast<uint4*>(O + (size_t)grow * (H * 128) + hu * 128 + cl * 8) = val;
+      }
+      // the next unit's first V may overwrite the staging area once every row is read back
+      fence_proxy_async_smem();
+      mbar_arrive(&sh->stage_free);
     } else {
-    // merge the two parities; parity 1 has tiles only when nj >= 2
+    // merge the two parities; parity 1 has tiles only when nt >= 2
     sh->xm[par][row] = m;
     sh->xl[par][row] = l;
     named_bar_sync(1 + quarter, 64);                // the even and the odd warp of this lane quarter
-    const bool two = nj >= 2;
+    const bool two = nt >= 2;
     const float m0v = sh->xm[0][row], m1v = sh->xm[1][row];
     const float mm = two ? fmaxf(m0v, m1v) : m0v;
     const float a0 = ex2_approx(m0v - mm);
@@ -530,6 +671,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     }
     }  // two-parity merge
+    }  // units
   }
 
   tc_fence_before();
@@ -537,7 +679,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tm, 512);
+    tmem_dealloc(tm, AttnCfg<kPar>::kCols);
   }
 }
 
@@ -547,6 +689,7 @@ __global__ void __launch_bounds__(256) k_attn_combine(const float* __restrict__ 
                                                       const float2* __restrict__ part_ml, int n_tail, int s_tail,
                                                       int u_full, int QT, int M, int H,
                                                       __nv_bfloat16* __restrict__ O) {
+  pdl_prologue();
   const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int tu = w / kAttnBM, row = w % kAttnBM;
   if (tu >= n_tail) return;
@@ -605,7 +748,7 @@ size_t tail_split_bytes(const TailSplit& p) {
 
 size_t attention_split_bytes(int M, int L, int H) {
   if (M <= 0 || L <= 0 || H <= 0) return 0;
-  if ((L + kAttnBN - 1) / kAttnBN <= kTwoQMaxTiles && M > kAttnBM) return 0;   // two-query-tile CTAs: no split
+  if ((L + kAttnBN - 1) / kAttnBN <= kShortMaxTiles) return 0;   // one-parity CTAs: no split
   const int QT = (M + kAttnBM - 1) / kAttnBM;
   return tail_split_bytes(plan_tail(QT * H, (L + kAttnBN - 1) / kAttnBN, num_sms()));
 }
@@ -626,23 +769,26 @@ int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, in
   if (rc) return rc;
   static PerContextOnce attr;
   rc = attr.ensure([](void**) {
-    if (cudaFuncSetAttribute(k_attn_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) !=
+    if (cudaFuncSetAttribute(k_attn_tc<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg<2>::kSmem) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(k_attn_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem) != cudaSuccess)
+        cudaFuncSetAttribute(k_attn_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg<1>::kSmem) !=
+            cudaSuccess)
       return check_launch("attention: shared-memory attribute");
     return (int)HSA_OK;
   });
   if (rc) return rc;
   const int nj_all = (L + kAttnBN - 1) / kAttnBN;
-  if (nj_all <= kTwoQMaxTiles && M > kAttnBM) {
-    // short key range: two query tiles per CTA share every K/V tile, no key-range split
-    const int QT2 = (M + 2 * kAttnBM - 1) / (2 * kAttnBM);
-    AttnGrid g{QT2, QT2 * H, 1, nullptr, nullptr};
+  if (nj_all <= kShortMaxTiles) {
+    // short key range: persistent one-parity CTAs, two per SM, each walking units blockIdx.x,
+    // blockIdx.x + grid, ... (all whole)
+    const int QT = (M + kAttnBM - 1) / kAttnBM, U = QT * H;
+    const int ctas = U < 2 * num_sms() ? U : 2 * num_sms();
+    AttnGrid g{QT, U, 1, nullptr, nullptr};
     ScopedTiming timing(HSA_KCLASS_ATTENTION, st);
-    k_attn_tc<true><<<QT2 * H, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, M, L, H,
-                                                               reinterpret_cast<__nv_bfloat16*>(O), g);
+    launch(k_attn_tc<1>, ctas, AttnCfg<1>::kThreads, AttnCfg<1>::kSmem, st, tq, tk, tv, M, L, H,
+           reinterpret_cast<__nv_bfloat16*>(O), g);
     count_launch(1);
-    return check_launch("attn_tc (two query tiles) launch");
+    return check_launch("attn_tc (one parity) launch");
   }
   const int QT = (M + kAttnBM - 1) / kAttnBM, U = QT * H;
   TailSplit ts = plan_tail(U, nj_all, num_sms());
@@ -656,15 +802,15 @@ int attention_bf16(const void* Q, int M, const void* K, const void* V, int L, in
   }
   ScopedTiming timing(HSA_KCLASS_ATTENTION, st);
   const int ctas = ts.u_full + ts.n_tail * ts.s_tail;
-  k_attn_tc<false><<<ctas, kAttnThreads, kAttnSmem, st>>>(tq, tk, tv, M, L, H, reinterpret_cast<__nv_bfloat16*>(O),
-                                                          g);
+  launch(k_attn_tc<2>, ctas, AttnCfg<2>::kThreads, AttnCfg<2>::kSmem, st, tq, tk, tv, M, L, H,
+         reinterpret_cast<__nv_bfloat16*>(O), g);
   count_launch(1);
   if (ts.s_tail > 1) {
     rc = check_launch("attn_tc launch");
     if (rc) return rc;
     const int warps = ts.n_tail * kAttnBM;
-    k_attn_combine<<<(warps + 7) / 8, 256, 0, st>>>(g.part_o, g.part_ml, ts.n_tail, ts.s_tail, ts.u_full, QT, M, H,
-                                                     reinterpret_cast<__nv_bfloat16*>(O));
+    launch(k_attn_combine, (warps + 7) / 8, 256, 0, st, g.part_o, g.part_ml, ts.n_tail, ts.s_tail, ts.u_full, QT, M,
+           H, reinterpret_cast<__nv_bfloat16*>(O));
     count_launch(1);
     return check_launch("attn_combine launch");
   }

@@ -38,6 +38,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of the library opens with this and is launched with programmatic stream
+// serialization (hsa::launch).  The wait returns once the grids ahead of this one in the stream
+// have completed and their memory writes are visible (at once when the launch carried no
+// programmatic dependency), so no kernel touches global memory early; what the launch gains is
+// that the grid is set up while its predecessor drains.  No kernel signals its dependents
+// early (griddepcontrol.launch_dependents): measured, that let the next kernel's CTAs sit on
+// the SMs in their wait while the current grid still ran, and slowed the small fp32 loop by 45 %.
+__device__ __forceinline__ void pdl_prologue() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

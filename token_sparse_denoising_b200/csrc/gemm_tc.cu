@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmY, int M, int Nout, int K, const float* __restrict__ bias,
               const float* __restrict__ gate, void* __restrict__ out) {
+  pdl_prologue();
   using Cfg = GemmCfg<BN>;
   constexpr int S = Cfg::kStages;
   constexpr bool kF32Out = (EPI == EPI_RESID || EPI == EPI_F32);
@@ -251,7 +252,7 @@ static int launch_gemm_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CU
   const int tiles = (Nout / BN) * ((M + kGemmBM - 1) / kGemmBM);
   dim3 grid(tiles < num_sms() ? tiles : num_sms());
   ScopedTiming timing(HSA_KCLASS_GEMM, st);
-  kern<<<grid, kGemmThreads, GemmCfg<BN>::kSmem, st>>>(ta, tb, ty, M, Nout, K, bias, gate, out);
+  launch(kern, grid, kGemmThreads, GemmCfg<BN>::kSmem, st, ta, tb, ty, M, Nout, K, bias, gate, out);
   count_launch(1);
   return check_launch("gemm_tc launch");
 }

@@ -7,6 +7,7 @@
 
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "../../include/hsa.h"
 
@@ -76,6 +77,24 @@ class ScopedTiming {
   cudaStream_t st_;
   cudaEvent_t a_ = nullptr;
 };
+
+// Launches `kernel` on `st` with programmatic stream serialization allowed, so its CTAs may
+// be scheduled while the kernel ahead of it finishes (each kernel's pdl_prologue keeps the
+// memory order).  A launch error is left for check_launch to report.
+template <typename... P, typename... A>
+void launch(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, A&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

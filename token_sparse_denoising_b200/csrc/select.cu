@@ -184,6 +184,7 @@ __device__ void radix_pass2(KeySource key, int N, const uint32_t* prefix, const 
 __global__ void __launch_bounds__(kSelectThreads, 1)
     k_select(const float* __restrict__ score, const uint8_t* __restrict__ pinned, int N, SelectArgs a,
              int8_t* __restrict__ group, int* __restrict__ order) {
+  pdl_prologue();
   __shared__ uint32_t hist[512];
   __shared__ int warp_sums[33];
   __shared__ int s_wcnt[kMaxGroups][kSelectThreads / 32];   // per group, per warp: count, then offset
@@ -409,7 +410,7 @@ extern "C" int hsa_select_tokens_pinned(const float* d_score, const uint8_t* d_p
   });
   if (arc) return arc;
   ScopedTiming timing(HSA_KCLASS_OTHER, as_stream(stream));
-  k_select<<<1, kSelectThreads, dyn, as_stream(stream)>>>(d_score, d_pinned, N, a, d_group, d_order);
+  launch(k_select, 1, kSelectThreads, dyn, as_stream(stream), d_score, d_pinned, N, a, d_group, d_order);
   count_launch(1);
   return check_launch("select launch");
 }
@@ -430,6 +431,7 @@ struct RowSegments {
 // M output positions; each finds its segment among at most 16.
 __global__ void __launch_bounds__(256) k_active_rows(const int32_t* __restrict__ order, RowSegments seg,
                                                      int32_t* __restrict__ idx) {
+  pdl_prologue();
   const int M = seg.dst[seg.n];
   for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < M; r += gridDim.x * blockDim.x) {
     int k = 0;
@@ -463,7 +465,7 @@ extern "C" int hsa_active_rows(const int32_t* d_order, int N, int K, const int* 
   if (pos == 0) return HSA_OK;
   if (!d_order || !d_idx) return set_error(HSA_EINVAL, "active_rows: null device pointer");
   const int blocks = (pos + 255) / 256 < 4 * num_sms() ? (pos + 255) / 256 : 4 * num_sms();
-  k_active_rows<<<blocks, 256, 0, as_stream(stream)>>>(d_order, seg, d_idx);
+  launch(k_active_rows, blocks, 256, 0, as_stream(stream), d_order, seg, d_idx);
   count_launch(1);
   return check_launch("active_rows launch");
 }

@@ -20,6 +20,7 @@ namespace hsa {
 template <typename T>
 __global__ void __launch_bounds__(256) k_row_sumsq(const T* __restrict__ in, int in_stride, int M, int D,
                                                    float* __restrict__ ss, int ss_stride) {
+  pdl_prologue();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= M) return;
@@ -44,6 +45,7 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope_ext(const T* __restrict__ 
                                                           const float* __restrict__ g_q,
                                                           const float* __restrict__ g_k, T* __restrict__ Q,
                                                           T* __restrict__ Kc, T* __restrict__ Vc) {
+  pdl_prologue();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= M) return;
@@ -79,6 +81,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_rms_rows_ext(const T* __restrict__ in, int in_stride, int M, int D,
                                                       float inv_d, const float* __restrict__ ss, int ss_stride,
                                                       const float* __restrict__ g, T* __restrict__ out) {
+  pdl_prologue();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= M) return;
@@ -98,6 +101,7 @@ __global__ void __launch_bounds__(256) k_rms_rows_ext(const T* __restrict__ in, 
 __global__ void __launch_bounds__(256) k_gated_residual(float* __restrict__ X, const float* __restrict__ y, int M,
                                                         int D, const float* __restrict__ b,
                                                         const float* __restrict__ gate) {
+  pdl_prologue();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= M) return;
@@ -154,11 +158,11 @@ extern "C" int hsa_row_sumsq(const void* d_in, int in_stride, int M, int D, int 
   cudaStream_t st = as_stream(stream);
   ScopedTiming timing(HSA_KCLASS_OTHER, st);
   if (dtype == HSA_BF16)
-    k_row_sumsq<__nv_bfloat16><<<shard_warp_blocks(M), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(d_in),
-                                                                    in_stride, M, D, d_ss, ss_stride);
+    launch(k_row_sumsq<__nv_bfloat16>, shard_warp_blocks(M), 256, 0, st,
+           static_cast<const __nv_bfloat16*>(d_in), in_stride, M, D, d_ss, ss_stride);
   else
-    k_row_sumsq<float><<<shard_warp_blocks(M), 256, 0, st>>>(static_cast<const float*>(d_in), in_stride, M, D, d_ss,
-                                                            ss_stride);
+    launch(k_row_sumsq<float>, shard_warp_blocks(M), 256, 0, st, static_cast<const float*>(d_in), in_stride, M, D,
+           d_ss, ss_stride);
   count_launch(1);
   return check_launch("row_sumsq launch");
 }
@@ -180,13 +184,12 @@ extern "C" int hsa_qk_norm_rope_ext(const void* d_qkv, int M, int N, int Dl, int
   const float inv_d = 1.0f / (float)D_total;
   if (dtype == HSA_BF16) {
     using T = __nv_bfloat16;
-    k_qk_norm_rope_ext<T><<<shard_warp_blocks(M), 256, 0, st>>>(
-        static_cast<const T*>(d_qkv), d_idx, d_pos, M, N, Dl, inv_d, d_ss, d_g_q, d_g_k, static_cast<T*>(d_Q),
-        static_cast<T*>(d_kcache), static_cast<T*>(d_vcache));
+    launch(k_qk_norm_rope_ext<T>, shard_warp_blocks(M), 256, 0, st, static_cast<const T*>(d_qkv), d_idx, d_pos, M, N,
+           Dl, inv_d, d_ss, d_g_q, d_g_k, static_cast<T*>(d_Q), static_cast<T*>(d_kcache), static_cast<T*>(d_vcache));
   } else {
-    k_qk_norm_rope_ext<float><<<shard_warp_blocks(M), 256, 0, st>>>(
-        static_cast<const float*>(d_qkv), d_idx, d_pos, M, N, Dl, inv_d, d_ss, d_g_q, d_g_k,
-        static_cast<float*>(d_Q), static_cast<float*>(d_kcache), static_cast<float*>(d_vcache));
+    launch(k_qk_norm_rope_ext<float>, shard_warp_blocks(M), 256, 0, st, static_cast<const float*>(d_qkv), d_idx, d_pos,
+           M, N, Dl, inv_d, d_ss, d_g_q, d_g_k, static_cast<float*>(d_Q), static_cast<float*>(d_kcache),
+           static_cast<float*>(d_vcache));
   }
   count_launch(1);
   return check_launch("qk_norm_rope_ext launch");
@@ -205,12 +208,11 @@ extern "C" int hsa_rms_rows_ext(const void* d_in, int in_stride, int M, int D, i
   const float inv_d = 1.0f / (float)D_total;
   if (dtype == HSA_BF16) {
     using T = __nv_bfloat16;
-    k_rms_rows_ext<T><<<shard_warp_blocks(M), 256, 0, st>>>(static_cast<const T*>(d_in), in_stride, M, D, inv_d, d_ss,
-                                                            ss_stride, d_g, static_cast<T*>(d_out));
+    launch(k_rms_rows_ext<T>, shard_warp_blocks(M), 256, 0, st, static_cast<const T*>(d_in), in_stride, M, D, inv_d,
+           d_ss, ss_stride, d_g, static_cast<T*>(d_out));
   } else {
-    k_rms_rows_ext<float><<<shard_warp_blocks(M), 256, 0, st>>>(static_cast<const float*>(d_in), in_stride, M, D,
-                                                                inv_d, d_ss, ss_stride, d_g,
-                                                                static_cast<float*>(d_out));
+    launch(k_rms_rows_ext<float>, shard_warp_blocks(M), 256, 0, st, static_cast<const float*>(d_in), in_stride, M, D,
+           inv_d, d_ss, ss_stride, d_g, static_cast<float*>(d_out));
   }
   count_launch(1);
   return check_launch("rms_rows_ext launch");
@@ -225,7 +227,7 @@ extern "C" int hsa_gated_residual(float* d_X, const float* d_y, int M, int D, co
     return set_error(HSA_EINVAL, "gated_residual: null or misaligned pointer");
   cudaStream_t st = as_stream(stream);
   ScopedTiming timing(HSA_KCLASS_OTHER, st);
-  k_gated_residual<<<shard_warp_blocks(M), 256, 0, st>>>(d_X, d_y, M, D, d_b, d_gate);
+  launch(k_gated_residual, shard_warp_blocks(M), 256, 0, st, d_X, d_y, M, D, d_b, d_gate);
   count_launch(1);
   return check_launch("gated_residual launch");
 }

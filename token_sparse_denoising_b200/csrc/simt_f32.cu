@@ -16,6 +16,7 @@ template <int EPI, int BM>
 __global__ void __launch_bounds__(256) k_gemm_f32(const float* __restrict__ A, const float* __restrict__ W, int M,
                                                   int Nout, int K, const float* __restrict__ bias,
                                                   const float* __restrict__ gate, float* __restrict__ out) {
+  pdl_prologue();
   constexpr int RM = BM / 16;                       // rows per thread
   __shared__ float As[16][BM + 4];
   __shared__ float Ws[16][68];
@@ -75,11 +76,11 @@ static void launch_gemm_f32(const float* A, int M, int K, const float* W, int No
   const long long nb = (Nout + 63) / 64, want = 2LL * num_sms();
   const auto blocks = [&](int bm) { return nb * ((M + bm - 1) / bm); };
   if (blocks(64) >= want) {
-    k_gemm_f32<EPI, 64><<<dim3((unsigned)nb, (M + 63) / 64), 256, 0, st>>>(A, W, M, Nout, K, bias, gate, out);
+    launch(k_gemm_f32<EPI, 64>, dim3((unsigned)nb, (M + 63) / 64), 256, 0, st, A, W, M, Nout, K, bias, gate, out);
   } else if (blocks(32) >= want) {
-    k_gemm_f32<EPI, 32><<<dim3((unsigned)nb, (M + 31) / 32), 256, 0, st>>>(A, W, M, Nout, K, bias, gate, out);
+    launch(k_gemm_f32<EPI, 32>, dim3((unsigned)nb, (M + 31) / 32), 256, 0, st, A, W, M, Nout, K, bias, gate, out);
   } else {
-    k_gemm_f32<EPI, 16><<<dim3((unsigned)nb, (M + 15) / 16), 256, 0, st>>>(A, W, M, Nout, K, bias, gate, out);
+    launch(k_gemm_f32<EPI, 16>, dim3((unsigned)nb, (M + 15) / 16), 256, 0, st, A, W, M, Nout, K, bias, gate, out);
   }
 }
 
@@ -113,6 +114,7 @@ __global__ void __launch_bounds__(256, 2) k_attn_f32(const float* __restrict__ Q
                                                      const float* __restrict__ V, int L, int H, int n_split,
                                                      float* __restrict__ O, float* __restrict__ part_o,
                                                      float2* __restrict__ part_ml) {
+  pdl_prologue();
   extern __shared__ float4 sm4[];
   float* Qs = reinterpret_cast<float*>(sm4);        // [32][132]
   float* Ks = Qs + kF32BQ * kF32Ld;                  // [64][132]
@@ -241,6 +243,7 @@ __global__ void __launch_bounds__(256, 2) k_attn_f32(const float* __restrict__ Q
 __global__ void __launch_bounds__(256) k_attn_f32_combine(const float* __restrict__ part_o,
                                                           const float2* __restrict__ part_ml, int M, int H,
                                                           int n_split, float* __restrict__ O) {
+  pdl_prologue();
   const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int QB = (M + kF32BQ - 1) / kF32BQ;
   const int row = w % kF32BQ, unit = w / kF32BQ;       // unit = h * QB + qb
@@ -305,12 +308,12 @@ int attention_f32(const float* Q, int M, const float* K, const float* V, int L, 
       S > 1 ? reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + align256(slots * 128 * sizeof(float))) : nullptr;
   if (S > 1 && align256(slots * 128 * sizeof(float)) + slots * sizeof(float2) > ws_bytes) S = 1;
   ScopedTiming timing(HSA_KCLASS_ATTENTION, st);
-  k_attn_f32<<<(unsigned)(QB * H * S), 256, kF32AttnSmem, st>>>(Q, M, K, V, L, H, S, O, part_o, part_ml);
+  launch(k_attn_f32, (unsigned)(QB * H * S), 256, kF32AttnSmem, st, Q, M, K, V, L, H, S, O, part_o, part_ml);
   count_launch(1);
   rc = check_launch("attn_f32 launch");
   if (rc || S == 1) return rc;
   const long long warps = (long long)QB * H * kF32BQ;
-  k_attn_f32_combine<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(part_o, part_ml, M, H, S, O);
+  launch(k_attn_f32_combine, (unsigned)((warps + 7) / 8), 256, 0, st, part_o, part_ml, M, H, S, O);
   count_launch(1);
   return check_launch("attn_f32 combine launch");
 }

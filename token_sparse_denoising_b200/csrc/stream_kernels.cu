@@ -55,37 +55,35 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
 }
 
 // ------------------------------------------------------------------ §2.3 cached Euler
-// x[e] += dsigma * v_hat[e] for every element; n4 float4 groups, grid-stride with
-// U groups per thread per iteration, all loaded before any is used.
+// x[e] += dsigma * v_hat[e] for every element; n4 float4 groups.  Each thread takes up to U
+// groups a grid-stride apart per pass, all loaded before any is used; the host sizes the grid
+// as a whole number of blocks per SM, so one pass is one balanced wave.
 __global__ void __launch_bounds__(256) k_euler(float* __restrict__ x, const float* __restrict__ vhat, size_t n4,
                                                float dsigma) {
+  pdl_prologue();
   constexpr int U = 4;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
-  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  for (; i + (U - 1) * stride < n4; i += U * stride) {
+  for (size_t base = (size_t)blockIdx.x * blockDim.x + threadIdx.x; base < n4; base += U * stride) {
     float4 xv[U], v[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      xv[u] = ld4_stream(x + 4 * (i + u * stride));
-      v[u] = ld4_stream(vhat + 4 * (i + u * stride));
+      const size_t i = base + u * stride;
+      if (i < n4) {
+        xv[u] = ld4_stream(x + 4 * i);
+        v[u] = ld4_stream(vhat + 4 * i);
+      }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      xv[u].x = fmaf(dsigma, v[u].x, xv[u].x);
-      xv[u].y = fmaf(dsigma, v[u].y, xv[u].y);
-      xv[u].z = fmaf(dsigma, v[u].z, xv[u].z);
-      xv[u].w = fmaf(dsigma, v[u].w, xv[u].w);
-      __stcs(reinterpret_cast<float4*>(x + 4 * (i + u * stride)), xv[u]);
+      const size_t i = base + u * stride;
+      if (i < n4) {
+        xv[u].x = fmaf(dsigma, v[u].x, xv[u].x);
+        xv[u].y = fmaf(dsigma, v[u].y, xv[u].y);
+        xv[u].z = fmaf(dsigma, v[u].z, xv[u].z);
+        xv[u].w = fmaf(dsigma, v[u].w, xv[u].w);
+        __stcs(reinterpret_cast<float4*>(x + 4 * i), xv[u]);
+      }
     }
-  }
-  for (; i < n4; i += stride) {
-    float4 xv = ld4_stream(x + 4 * i);
-    const float4 v = ld4_stream(vhat + 4 * i);
-    xv.x = fmaf(dsigma, v.x, xv.x);
-    xv.y = fmaf(dsigma, v.y, xv.y);
-    xv.z = fmaf(dsigma, v.z, xv.z);
-    xv.w = fmaf(dsigma, v.w, xv.w);
-    __stcs(reinterpret_cast<float4*>(x + 4 * i), xv);
   }
 }
 
@@ -96,6 +94,7 @@ __global__ void __launch_bounds__(256) k_scatter_vhat(float* __restrict__ vhat, 
                                                       const int* __restrict__ idx, int M, int N, int C,
                                                       float* __restrict__ score, float* __restrict__ x,
                                                       float dsigma) {
+  pdl_prologue();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= M) return;
@@ -152,6 +151,7 @@ __global__ void __launch_bounds__(256) k_scatter_vhat(float* __restrict__ vhat, 
 // §2.1 score on its own: score[n] = sum|v_new - v_prev| / (sum|v_prev| + eps).
 __global__ void __launch_bounds__(256) k_l1_score(const float* __restrict__ vnew, const float* __restrict__ vprev,
                                                   int N, int C, float* __restrict__ score) {
+  pdl_prologue();
   const int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (n >= N) return;
@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(256) k_ln_rows(float* __restrict__ X, const fl
                                                  const int* __restrict__ idx, int M, int N,
                                                  const float* __restrict__ mul, const float* __restrict__ add,
                                                  int mul_plus_one, TOut* __restrict__ h) {
+  pdl_prologue();
   constexpr int D = VPT * 128;
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -231,6 +232,7 @@ __global__ void __launch_bounds__(256) k_ln_rows_any(float* __restrict__ X, cons
                                                      const int* __restrict__ idx, int M, int N, int D,
                                                      const float* __restrict__ mul, const float* __restrict__ add,
                                                      int mul_plus_one, TOut* __restrict__ h) {
+  pdl_prologue();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= M) return;
@@ -301,6 +303,7 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope(const TIn* __restrict__ qk
                                                       const float* __restrict__ g_q, const float* __restrict__ g_k,
                                                       TOut* __restrict__ Q, TOut* __restrict__ Kc,
                                                       TOut* __restrict__ Vc) {
+  pdl_prologue();
   constexpr int D = VPT * 128;
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -354,6 +357,7 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope(const TIn* __restrict__ qk
 template <typename TIn, typename TOut>
 __global__ void __launch_bounds__(256) k_rms_rows(const TIn* __restrict__ in, int in_stride, int M, int D,
                                                   const float* __restrict__ g, TOut* __restrict__ out) {
+  pdl_prologue();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= M) return;
@@ -385,6 +389,7 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope_any(const TIn* __restrict_
                                                           const float* __restrict__ g_q,
                                                           const float* __restrict__ g_k, TOut* __restrict__ Q,
                                                           TOut* __restrict__ Kc, TOut* __restrict__ Vc) {
+  pdl_prologue();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= M) return;
@@ -425,6 +430,7 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope_any(const TIn* __restrict_
 template <typename TOut>
 __global__ void __launch_bounds__(256) k_gather_rows(const float* __restrict__ x, const int* __restrict__ idx, int M,
                                                      int N, int C, TOut* __restrict__ out) {
+  pdl_prologue();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= M) return;
