@@ -56,12 +56,14 @@ def parse():
     p.add_argument("--no-configs", action="store_true",
                    help="skip the other workloads measured beside the headline (tiny loop, 30-block loop, "
                         "Wan-14B block, attention and Euler sweeps)")
-    p.add_argument("--mode", choices=["step", "loop", "sweep", "wan14", "tiny", "headpar", "cross"], default="step",
+    p.add_argument("--mode", choices=["step", "loop", "sweep", "wan14", "tiny", "headpar", "cross", "gemm"],
+                   default="step",
                    help="step: the headline line; loop: 30-block Wan-1.3B loop, HSA vs uniform 40 steps; "
                         "sweep: attention + Euler kernel sweep; wan14: Wan-14B block active-fraction sweep; "
                         "tiny: the fp32 parity workload as a whole run; headpar: one Wan-14B block split by "
                         "heads over the ranks (NCCL between the phases), |A|/N = 1; cross: the "
-                        "cross-attention shape alone (32760 queries x 512 context rows)")
+                        "cross-attention shape alone (32760 queries x 512 context rows); gemm: the block's "
+                        "GEMMs alone against cuBLAS")
     return p.parse_args()
 
 
@@ -592,16 +594,66 @@ def measure_cross(reps: int = 20, gen=None):
     return {"M": M, "L": L, "H": 12, "ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_burst": round(tf / peak_burst, 3)}
 
 
+def measure_gemm(gen=None, reps: int = 20):
+    """The Wan-1.3B block's GEMMs at |A|/N = 1 (M = 32760), each alone: the library's tcgen05 kernel
+    with its fused epilogue against cuBLAS (torch.nn.functional.linear, bf16 out, no epilogue) on
+    the same inputs, back to back; the working sets exceed L2."""
+    import torch
+    from token_sparse_denoising_b200 import hsa
+    hsa.load()
+    _, peak_burst, _, _ = load_peaks()
+    if gen is None:
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(5)
+    M, D, F = S.WAN13_GRID.N, S.WAN13_BLOCK.D, S.WAN13_BLOCK.F
+    out = []
+    # the residual GEMMs also with the plain bf16 store, the epilogue cuBLAS is timed with
+    for name, kin, nout, epi in (("qkv", D, 3 * D, hsa.EPI_STORE), ("o_proj", D, D, hsa.EPI_RESID),
+                                 ("o_proj_store", D, D, hsa.EPI_STORE), ("ffn1_gelu", D, F, hsa.EPI_GELU),
+                                 ("ffn2", F, D, hsa.EPI_RESID), ("ffn2_store", F, D, hsa.EPI_STORE)):
+        x = S.device_normal(gen, (M, kin), 1.0, True, "cuda")
+        w = S.device_normal(gen, (nout, kin), 0.02, True, "cuda")
+        b = torch.zeros(nout, device="cuda")
+        gate = torch.full((nout,), 0.5, device="cuda")
+        resid = epi == hsa.EPI_RESID
+        y = torch.zeros((M, nout), device="cuda") if resid else torch.empty((M, nout), dtype=torch.bfloat16,
+                                                                              device="cuda")
+        run = lambda: hsa.linear(x, w, b, epi, y, gate=gate if resid else None)
+        ref = lambda: torch.nn.functional.linear(x, w)
+        for _ in range(3):
+            run()
+            ref()
+        ms = time_device(run, reps, lambda: None) / reps
+        ms_ref = time_device(ref, reps, lambda: None) / reps
+        flop = 2.0 * M * kin * nout
+        out.append({"gemm": name, "M": M, "K": kin, "N": nout, "ms": round(ms, 4),
+                    "tflops": round(flop / (ms * 1e-3) / 1e12, 1),
+                    "frac_of_burst": round(flop / (ms * 1e-3) / 1e12 / peak_burst, 3),
+                    "cublas_ms": round(ms_ref, 4), "vs_cublas": round(ms_ref / ms, 3),
+                    "epilogue": {0: "bias, bf16 out", 1: "bias + GELU, bf16 out",
+                                 2: "fp32 residual += gate * (acc + bias), TMA reduce-add"}[epi]})
+        del x, w, y
+    assert hsa.device_status() == 0
+    torch.cuda.empty_cache()
+    return out
+
+
 def measure_sweep(reps: int = 5):
-    """Attention at N in {8190, 32760, 75600} x |A|/N in {1, .5, .25, .125} (12 heads, bf16 Q/K/V
-    N(0,1)) and the Euler update on N x 64 fp32 latents with the L2 flushed before each launch."""
+    """The cross-attention shape and the block's GEMMs (against cuBLAS), attention at N in {8190,
+    32760, 75600} x |A|/N in {1, .5, .25, .125} (12 heads, bf16 Q/K/V N(0,1)), and the Euler update
+    on N x 64 fp32 latents: one launch after an L2 flush, and back to back in one CUDA graph."""
     import torch
     from token_sparse_denoising_b200 import hsa
     hsa.load()
     _, peak_burst, hbm, src = load_peaks()
-    res = {"attention": [], "euler": [], "peaks": f"{src}: burst bf16 {peak_burst} TFLOP/s, HBM {hbm} GB/s"}
+    res = {"attention": [], "euler": [], "peaks": f"{src}: burst bf16 {peak_burst} TFLOP/s, HBM {hbm} GB/s",
+           "order": "cross-attention and GEMMs first, then the attention sweep, then the Euler update (the "
+                    "long attention launches hold the GPU at its power cap, which lowers the clock of "
+                    "whatever follows)"}
     gen = torch.Generator(device="cuda")
     gen.manual_seed(5)
+    res["cross_attention"] = measure_cross(4 * reps, gen)
+    res["gemm"] = measure_gemm(gen)
     for N in (8190, 32760, 75600):
         k = S.device_normal(gen, (N, 1536), 1.0, True, "cuda")
         v = S.device_normal(gen, (N, 1536), 1.0, True, "cuda")
@@ -632,7 +684,6 @@ def measure_sweep(reps: int = 5):
                                        f"value = query_row_ms x {N} (the |A|/N = 1 launch)"}
             del kh, vh_
         del k, v
-    res["cross_attention"] = measure_cross(4 * reps, gen)
     flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda")      # 256 MB > L2: evicts between launches
     flush_r = torch.zeros(256 * 1024 * 1024 // 4, device="cuda")
     for N in (8190, 32760, 75600):
@@ -1006,7 +1057,8 @@ def main():
     if args.mode != "step":
         if rank == 0:
             fn = {"loop": run_loop, "sweep": run_sweep, "wan14": run_wan14, "tiny": run_tiny,
-                  "cross": lambda a: {"mode": "cross", **measure_cross()}}[args.mode]
+                  "cross": lambda a: {"mode": "cross", **measure_cross()},
+                  "gemm": lambda a: {"mode": "gemm", "gemm": measure_gemm()}}[args.mode]
             print(json.dumps(fn(args)), flush=True)
         return 0
     dist = None
