@@ -571,9 +571,10 @@ def measure_tiny(with_oracle: bool = True, reps: int = 5):
     return out
 
 
-def measure_cross(reps: int = 20, gen=None):
+def measure_cross(reps: int = 100, gen=None):
     """The cross-attention shape alone: every active query of the Wan-1.3B block (32760) against
-    the 512-row text context, 12 heads, bf16; two warm-up launches, then `reps` timed back to back."""
+    the 512-row text context, 12 heads, bf16; 30 warm-up launches (the clock settles from idle over
+    a few milliseconds), then `reps` timed back to back."""
     import torch
     from token_sparse_denoising_b200 import hsa
     hsa.load()
@@ -586,7 +587,7 @@ def measure_cross(reps: int = 20, gen=None):
     v = S.device_normal(gen, (L, 1536), 1.0, True, "cuda")
     q = S.device_normal(gen, (M, 1536), 1.0, True, "cuda")
     o = torch.empty_like(q)
-    for _ in range(2):
+    for _ in range(30):
         hsa.attention(q, k, v, 12, o)
     ms = time_device(lambda: hsa.attention(q, k, v, 12, o), reps, lambda: None) / reps
     tf = 4.0 * M * L * 128 * 12 / (ms * 1e-3) / 1e12
@@ -620,7 +621,7 @@ def measure_gemm(gen=None, reps: int = 20):
                                                                               device="cuda")
         run = lambda: hsa.linear(x, w, b, epi, y, gate=gate if resid else None)
         ref = lambda: torch.nn.functional.linear(x, w)
-        for _ in range(3):
+        for _ in range(10):
             run()
             ref()
         ms = time_device(run, reps, lambda: None) / reps
@@ -652,7 +653,7 @@ def measure_sweep(reps: int = 5):
                     "whatever follows)"}
     gen = torch.Generator(device="cuda")
     gen.manual_seed(5)
-    res["cross_attention"] = measure_cross(4 * reps, gen)
+    res["cross_attention"] = measure_cross(gen=gen)
     res["gemm"] = measure_gemm(gen)
     for N in (8190, 32760, 75600):
         k = S.device_normal(gen, (N, 1536), 1.0, True, "cuda")

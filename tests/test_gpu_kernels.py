@@ -63,8 +63,13 @@ def _select_case(seed, N, K, kind):
 
 @pytest.mark.parametrize("seed,N,K,kind", [(0, 1, 1, "rand"), (1, 5, 3, "ties"), (2, 1000, 2, "rand"),
                                            (3, 1000, 4, "ties"), (4, 4097, 5, "const"), (5, 32760, 3, "rand"),
-                                           (6, 32760, 16, "ties"), (7, 75600, 3, "rand")])
+                                           (6, 32760, 16, "ties"), (7, 75600, 3, "rand"), (8, 75600, 3, "const"),
+                                           (9, 300000, 3, "ties")])
 def test_select_tokens_bit_exact(cuda_lib, seed, N, K, kind):
+    """Bit-exact against the oracle.  The selection spreads N over the 8 CTAs of a cluster in ranges of
+    whole 1024-index blocks: one token, fewer tokens than one CTA's range (CTAs with nothing),
+    ragged ranges, all-equal scores (every boundary decided by token index across CTAs), up to 16
+    groups, and N = 300000, where each CTA's range exceeds what it stages in shared memory."""
     scores, sizes = _select_case(seed, N, K, kind)
     if seed == 5:
         sizes = S.group_sizes(N, (0.25, 0.25, 0.5))

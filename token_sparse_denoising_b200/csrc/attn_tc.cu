@@ -76,9 +76,8 @@ constexpr uint32_t kColS = 0;
 #define HSA_ATTN_POLY_PER8 0
 #endif
 constexpr int kPolyPer8 = HSA_ATTN_POLY_PER8;
-#ifndef HSA_ATTN_POLY_SHORT_PER8
-#define HSA_ATTN_POLY_SHORT_PER8 0
-#endif
+// The one-parity kernel of short key ranges measured the same way at the cross-attention shape
+// (32760 x 512, 12 heads): 0 / 2 / 4 of 8 took 0.132 / 0.133 / 0.143 ms, so it uses the MUFU path too.
 // P goes to the MMA warp in two halves of 64 keys; PV of the first half starts while the
 // softmax warps compute the exponentials of the second.  Measured at the Wan-1.3B shape
 // (attention alone): one release per tile 5.40 ms, halves 5.21 ms, quarters 5.47 ms.
@@ -517,8 +516,7 @@ __global__ void __launch_bounds__(AttnCfg<kPar>::kThreads, 3 - kPar)
 #pragma unroll
         for (int c = hh * 64; c < hh * 64 + 64; c += 2) {
           const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
-          // compile-time per unrolled column pair
-          const bool poly = (c & 7) >= 8 - (kPar == 1 ? HSA_ATTN_POLY_SHORT_PER8 : kPolyPer8);
+          const bool poly = (c & 7) >= 8 - kPolyPer8;  // compile-time per unrolled column pair
           const float p0 = poly ? ex2_poly(x.x) : ex2_approx(x.x);
           const float p1 = poly ? ex2_poly(x.y) : ex2_approx(x.y);
           rs4[(c >> 1) & 3] = fadd2(rs4[(c >> 1) & 3], make_float2(p0, p1));

@@ -10,23 +10,29 @@
 // [c_{k-1}, c_k) with c_k = n_1 + ... + n_k.  The result is unique, so the GPU
 // output is compared bit for bit.
 //
-// One 1024-thread CTA (the work is a few passes over N floats):
+// One cluster of 8 CTAs of 1024 threads (one CTA below 4096 tokens, where the cluster's barriers
+// cost more than they save).  CTA r of the cluster owns a contiguous range of token indices, and
+// warp w of a CTA a contiguous sub-range:
 //   1. for each boundary c_k (k < K): radix-select, over the 32-bit order key,
 //      the element of rank c_k - 1 (4 passes of 8 bits; per-warp private
-//      shared-memory histograms, since scores share few exponent bytes).  The
-//      top-digit pass is shared by all boundaries, and each later pass serves
-//      two boundaries at once: their key subsets are disjoint or identical, so
-//      one sweep fills both histograms.  Then the right index among the equal
-//      keys by a block scan;
+//      shared-memory histograms, since scores share few exponent bytes, summed
+//      per CTA and then over the cluster through distributed shared memory, so
+//      every CTA takes the same decision).  The top-digit pass is shared by all
+//      boundaries, and each later pass serves two boundaries at once: their key
+//      subsets are disjoint or identical, so one sweep fills both histograms.
+//      Then the right index among the equal keys by a scan over the warps and the
+//      CTAs; the CTA holding it publishes it to all;
 //   2. each token's group = number of boundaries it ranks at or after;
-//   3. the groups' lists, each ascending by index: warp w owns a contiguous index
-//      range and walks it 32 consecutive indices at a time (bank-conflict-free
-//      shared-memory reads, coalesced writes); per-group warp counts come from
-//      ballots, one scan over the warps per group gives each warp its offsets,
-//      and a lane's position is the number of lower lanes in its group.  Group k
-//      starts at c_{k-1}.
-// For N <= 36864 the order keys are first staged in shared memory, so the passes
-// do not wait on L2 latency for every element.
+//   3. the groups' lists, each ascending by index: each warp walks its range 32
+//      consecutive indices at a time (bank-conflict-free shared-memory reads,
+//      coalesced writes); per-group warp counts come from ballots, a scan over the
+//      warps and one over the CTAs give each warp its offsets, and a lane's
+//      position is the number of lower lanes in its group.  Group k starts at
+//      c_{k-1}.
+// Every CTA runs the same sequence of cluster barriers whatever the data, and the last
+// one keeps every CTA's shared memory alive until its peers have read it.
+// Up to 36864 keys per CTA are first staged in shared memory, so the passes do not wait
+// on L2 latency for every element.
 //
 // Also here: k_active_rows, which builds A_i from the group lists when the active
 // groups are not a prefix of the order (non-nested budgets).
@@ -35,15 +41,48 @@
 namespace hsa {
 
 constexpr int kSelectThreads = 1024;
+constexpr int kSelectCluster = 8;          // CTAs per cluster from kSelectClusterMinN tokens on
+constexpr int kSelectClusterMinN = 4096;   // below it one CTA (measured: N = 1024 13 us alone, 19 in a cluster)
 constexpr int kMaxGroups = 16;
 
-// Largest N whose keys are staged in shared memory (4 bytes each, on top of ~70 KB of
-// histograms); larger N reads the scores from global memory on every pass.
+// Most keys one CTA stages in shared memory (4 bytes each, on top of ~70 KB of histograms);
+// a CTA with a longer range reads the scores from global memory on every pass.
 constexpr int kSelectStagedMax = 36864;
+
+// ---- cluster helpers: rank, distributed shared memory, barrier
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+  return n;
+}
+// address of the same shared-memory variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t peer_smem(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ uint32_t ld_peer(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_peer(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// every thread of every CTA of the cluster; orders the shared-memory writes before it
+// (local and remote) before the reads after it
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 struct SelectArgs {
   int K;
-  int staged;               // 1: keys staged in dynamic shared memory
+  int staged;               // 1: each CTA's keys staged in dynamic shared memory
   int cum[kMaxGroups + 1];  // cum[0] = 0, cum[k] = n_1 + ... + n_k
 };
 
@@ -97,9 +136,10 @@ __device__ __forceinline__ uint32_t inverted_key(const float* __restrict__ score
 struct KeySource {
   const float* __restrict__ score;
   const uint8_t* __restrict__ pinned;  // nullable
-  const uint32_t* ikeys;               // shared memory, or nullptr
+  const uint32_t* ikeys;               // shared memory (this CTA's range from index lo), or nullptr
+  int lo;
   __device__ __forceinline__ uint32_t operator()(int n) const {
-    return ikeys ? ikeys[n] : inverted_key(score, pinned, n);
+    return ikeys ? ikeys[n - lo] : inverted_key(score, pinned, n);
   }
 };
 
@@ -136,15 +176,18 @@ __device__ __forceinline__ void scan_bins(const uint32_t* bins, int rank, int* o
 
 // One radix pass for nt <= 2 targets t, each a (prefix, mask) of the keys already fixed and the rank
 // sought among them: the histogram of the 8-bit digit at `shift` of every target's keys (per-warp
-// private copies, then summed), then, by warp t, target t's digit and the rank within that digit.
+// private copies over this CTA's indices [lo, hi), summed into hpub, then summed over the cluster's
+// CTAs into hist), then, by warp t, target t's digit and the rank within that digit.
 // Two targets select either disjoint key sets (different prefixes: bins [0,256) and [256,512)) or the
 // same one (equal prefix and mask: both read bins [0,256)), so one sweep over the keys serves both.
-// Every thread of the block calls it; hist keeps the summed bins for the caller.  NT is a template
+// Every thread of every CTA of the cluster calls it with the same targets; hist keeps the summed bins
+// for the caller.  Consecutive passes alternate between two hpub buffers: the cluster barrier of
+// the next pass keeps any CTA from rewriting a buffer its peers are still reading.  NT is a template
 // parameter so the single-target pass carries no second-target test per key.
 template <int NT>
-__device__ void radix_pass2(KeySource key, int N, const uint32_t* prefix, const uint32_t* mask,
-                            const int* rank, int shift, uint32_t (*hw)[kHistStride], uint32_t* hist,
-                            int* out_digit, int* out_rank) {
+__device__ void radix_pass2(KeySource key, int lo, int hi, const uint32_t* prefix, const uint32_t* mask,
+                            const int* rank, int shift, uint32_t (*hw)[kHistStride], uint32_t* hpub,
+                            uint32_t* hist, int* out_digit, int* out_rank) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int nt = NT;
   const bool shared_keys = NT == 2 && prefix[0] == prefix[1] && mask[0] == mask[1];
@@ -156,10 +199,10 @@ __device__ void radix_pass2(KeySource key, int N, const uint32_t* prefix, const 
   __syncwarp();
   // Keys of similar scores share their top bytes, so most lanes of a warp often carry the
   // same bin: the lanes equal to lane 0's bin add with one atomic, the rest one each.
-  for (int base = 0; base < N; base += kSelectThreads) {
+  for (int base = lo; base < hi; base += kSelectThreads) {
     const int n = base + tid;
     uint32_t bin = 0xFFFFu;                         // no contribution
-    if (n < N) {
+    if (n < hi) {
       const uint32_t ik = key(n);
       if ((ik & m0) == p0) bin = (ik >> shift) & 255u;
       else if (two && (ik & m1) == p1) bin = 256u + ((ik >> shift) & 255u);
@@ -174,6 +217,13 @@ __device__ void radix_pass2(KeySource key, int N, const uint32_t* prefix, const 
     uint32_t t = 0;
 #pragma unroll 8
     for (int w = 0; w < kSelectThreads / 32; ++w) t += hw[w][tid];
+    hpub[tid] = t;
+  }
+  cluster_sync();
+  if (tid < nbins) {
+    uint32_t t = 0;
+    const int nc = (int)cluster_size();
+    for (int q = 0; q < nc; ++q) t += ld_peer(peer_smem(hpub + tid, (uint32_t)q));
     hist[tid] = t;
   }
   __syncthreads();
@@ -186,31 +236,39 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
              int8_t* __restrict__ group, int* __restrict__ order) {
   pdl_prologue();
   __shared__ uint32_t hist[512];
+  __shared__ uint32_t hpub[2][512];                        // this CTA's pass histogram, for its peers
   __shared__ int warp_sums[33];
   __shared__ int s_wcnt[kMaxGroups][kSelectThreads / 32];   // per group, per warp: count, then offset
+  __shared__ int s_tcnt[kMaxGroups];                        // per boundary: this CTA's matching keys
+  __shared__ int s_gcnt[kMaxGroups];                        // per group: this CTA's tokens
   __shared__ uint32_t s_thr_key[kMaxGroups];
   __shared__ int s_thr_idx[kMaxGroups];
   __shared__ uint32_t s_pref[kMaxGroups], s_mask[kMaxGroups];   // per inner boundary (compacted list)
   __shared__ int s_rank[kMaxGroups], s_bnd[kMaxGroups];
   __shared__ int s_digit2[2], s_rank2[2];
-  // dynamic shared memory: the per-warp private histograms, then the N staged keys when the launch
-  // provides them
+  // dynamic shared memory: the per-warp private histograms, then this CTA's staged keys when the
+  // launch provides them
   extern __shared__ uint32_t s_dyn[];
   uint32_t (*hw)[kHistStride] = reinterpret_cast<uint32_t (*)[kHistStride]>(s_dyn);
   uint32_t* s_ikeys = s_dyn + (kSelectThreads / 32) * kHistStride;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int kWarps = kSelectThreads / 32;
-  // warp w owns indices [wlo, whi): a multiple of 32 per warp, walked 32 consecutive at a time
-  const int per_warp = ((N + kWarps * 32 - 1) / (kWarps * 32)) * 32;
-  const int wlo = min(N, warp * per_warp), whi = min(N, wlo + per_warp);
+  const int r = (int)cluster_rank(), nc = (int)cluster_size();
+  // CTA r owns indices [lo, hi), warp w [wlo, whi) within them: multiples of 32 per warp, walked
+  // 32 consecutive at a time
+  const int per_cta = ((N + nc * kWarps * 32 - 1) / (nc * kWarps * 32)) * kWarps * 32;
+  const int lo = min(N, r * per_cta), hi = min(N, lo + per_cta);
+  const int per_warp = per_cta / kWarps;
+  const int wlo = min(hi, lo + warp * per_warp), whi = min(hi, wlo + per_warp);
   const unsigned lanes_below = (1u << lane) - 1u;
-  KeySource key{score, pinned, nullptr};
+  KeySource key{score, pinned, nullptr, lo};
   if (a.staged) {
-    for (int n = tid; n < N; n += kSelectThreads) s_ikeys[n] = inverted_key(score, pinned, n);
+    for (int n = lo + tid; n < hi; n += kSelectThreads) s_ikeys[n - lo] = inverted_key(score, pinned, n);
     __syncthreads();
     key.ikeys = s_ikeys;
   }
+  int pass = 0;                                            // alternates the hpub buffers
 
   // ---- 1. threshold element of every inner boundary.  Ascending order of ik = ~key is descending
   // score order; boundary c_b needs the element of rank c_b - 1.  Boundaries with c_b <= 0 or
@@ -231,7 +289,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
   __syncthreads();
   if (nb > 0) {
     // top byte: one histogram serves every boundary
-    radix_pass2<1>(key, N, s_pref, s_mask, s_rank, 24, hw, hist, s_digit2, s_rank2);
+    radix_pass2<1>(key, lo, hi, s_pref, s_mask, s_rank, 24, hw, hpub[pass++ & 1], hist, s_digit2, s_rank2);
     if (warp == 0) {
       for (int i = 0; i < nb; ++i) {
         scan_bins(hist, s_rank[i], s_digit2, s_rank2);
@@ -249,10 +307,11 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
   for (int i0 = 0; i0 < nb; i0 += 2) {
     const int nt = nb - i0 < 2 ? nb - i0 : 2;
     for (int shift = 16; shift >= 0; shift -= 8) {
+      uint32_t* hp = hpub[pass++ & 1];
       if (nt == 2)
-        radix_pass2<2>(key, N, s_pref + i0, s_mask + i0, s_rank + i0, shift, hw, hist, s_digit2, s_rank2);
+        radix_pass2<2>(key, lo, hi, s_pref + i0, s_mask + i0, s_rank + i0, shift, hw, hp, hist, s_digit2, s_rank2);
       else
-        radix_pass2<1>(key, N, s_pref + i0, s_mask + i0, s_rank + i0, shift, hw, hist, s_digit2, s_rank2);
+        radix_pass2<1>(key, lo, hi, s_pref + i0, s_mask + i0, s_rank + i0, shift, hw, hp, hist, s_digit2, s_rank2);
       if (tid < nt) {
         s_pref[i0 + tid] |= (uint32_t)s_digit2[tid] << shift;
         s_mask[i0 + tid] |= 255u << shift;
@@ -261,10 +320,12 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
       __syncthreads();
     }
     for (int t = 0; t < nt; ++t) {
-      const uint32_t prefix = s_pref[i0 + t];
-      const int rank = s_rank[i0 + t], b = s_bnd[i0 + t];
+      const int i = i0 + t;
+      const uint32_t prefix = s_pref[i];
+      const int rank = s_rank[i], b = s_bnd[i];
       // the rank-th smallest token index among keys equal to the target: per-warp counts of
-      // matches, a scan over the warps, then the warp holding that rank finds the lane
+      // matches, scans over the warps and over the CTAs, then the warp holding that rank finds the
+      // lane and hands the threshold to every CTA of the cluster
       int cnt = 0;
       for (int base = wlo; base < whi; base += 32) {
         const int n = base + lane;
@@ -281,9 +342,12 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
           if (lane >= o) incl += y;
         }
         warp_sums[lane] = incl - v;
+        if (lane == 31) s_tcnt[i] = incl;                  // this CTA's matches
       }
-      __syncthreads();
-      const int excl = warp_sums[warp];
+      cluster_sync();
+      int cta_excl = 0;
+      for (int q = 0; q < r; ++q) cta_excl += (int)ld_peer(peer_smem(s_tcnt + i, (uint32_t)q));
+      const int excl = cta_excl + warp_sums[warp];
       if (rank >= excl && rank < excl + cnt) {      // warp-uniform
         int seen = excl;
         for (int base = wlo; base < whi; base += 32) {
@@ -292,15 +356,17 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
           const unsigned mk = __ballot_sync(0xffffffffu, m);
           if (rank < seen + __popc(mk)) {
             if (m && seen + __popc(mk & lanes_below) == rank) {
-              s_thr_idx[b] = n;
-              s_thr_key[b] = ~prefix;
+              for (int q = 0; q < nc; ++q) {
+                st_peer(peer_smem(s_thr_idx + b, (uint32_t)q), (uint32_t)n);
+                st_peer(peer_smem(s_thr_key + b, (uint32_t)q), ~prefix);
+              }
             }
             break;
           }
           seen += __popc(mk);
         }
       }
-      __syncthreads();
+      cluster_sync();
     }
   }
 
@@ -329,7 +395,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
         }
       }
       group[n] = (int8_t)g;
-      if (key.ikeys) s_ikeys[n] = (uint32_t)g;   // this lane's own slot: it now holds the group
+      if (key.ikeys) s_ikeys[n - lo] = (uint32_t)g;   // this lane's own slot: it now holds the group
     }
 #pragma unroll
     for (int k = 0; k < kMaxGroups; ++k)
@@ -341,16 +407,24 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
       if (k < a.K) s_wcnt[k][warp] = cnt[k];
   }
   __syncthreads();
-  // ---- 3. offsets: warp k scans group k's counts over the warps (ascending index ranges)
+  // ---- 3. offsets: warp k scans group k's counts over the warps (ascending index ranges), then
+  // adds the counts of the CTAs with lower index ranges
+  int incl_k = 0, v_k = 0;
   if (warp < a.K) {
-    const int v = s_wcnt[warp][lane];
-    int incl = v;
+    v_k = s_wcnt[warp][lane];
+    incl_k = v_k;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+      const int y = __shfl_up_sync(0xffffffffu, incl_k, o);
+      if (lane >= o) incl_k += y;
     }
-    s_wcnt[warp][lane] = a.cum[warp] + incl - v;
+    if (lane == 31) s_gcnt[warp] = incl_k;               // this CTA's tokens of group `warp`
+  }
+  cluster_sync();
+  if (warp < a.K) {
+    int cta_off = 0;
+    for (int q = 0; q < r; ++q) cta_off += (int)ld_peer(peer_smem(s_gcnt + warp, (uint32_t)q));
+    s_wcnt[warp][lane] = a.cum[warp] + cta_off + incl_k - v_k;
   }
   __syncthreads();
   int off[kMaxGroups];
@@ -358,7 +432,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
   for (int k = 0; k < kMaxGroups; ++k) off[k] = (k < a.K) ? s_wcnt[k][warp] : 0;
   for (int base = wlo; base < whi; base += 32) {
     const int n = base + lane;
-    const int g = n < whi ? (key.ikeys ? (int)s_ikeys[n] : (int)group[n]) : -1;
+    const int g = n < whi ? (key.ikeys ? (int)s_ikeys[n - lo] : (int)group[n]) : -1;
 #pragma unroll
     for (int k = 0; k < kMaxGroups; ++k) {
       if (k < a.K) {
@@ -368,6 +442,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1)
       }
     }
   }
+  // no CTA leaves while a peer may still read its shared memory
+  cluster_sync();
 }
 
 }  // namespace hsa
@@ -398,9 +474,12 @@ extern "C" int hsa_select_tokens_pinned(const float* d_score, const uint8_t* d_p
   }
   if (c != N) return set_error(HSA_EINVAL, "select: group sizes must sum to N");
   if (N == 0) return HSA_OK;
-  a.staged = N <= kSelectStagedMax ? 1 : 0;
+  // cluster size, and each CTA's index range as the kernel computes it
+  const int nc = N < kSelectClusterMinN ? 1 : kSelectCluster;
+  const int per_cta = (N + nc * kSelectThreads - 1) / (nc * kSelectThreads) * kSelectThreads;
+  a.staged = per_cta <= kSelectStagedMax ? 1 : 0;
   constexpr size_t kHistBytes = (size_t)(kSelectThreads / 32) * kHistStride * sizeof(uint32_t);
-  const size_t dyn = kHistBytes + (a.staged ? (size_t)N * sizeof(uint32_t) : 0);
+  const size_t dyn = kHistBytes + (a.staged ? (size_t)per_cta * sizeof(uint32_t) : 0);
   static PerContextOnce attr;
   const int arc = attr.ensure([](void**) {
     if (cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -410,7 +489,11 @@ extern "C" int hsa_select_tokens_pinned(const float* d_score, const uint8_t* d_p
   });
   if (arc) return arc;
   ScopedTiming timing(HSA_KCLASS_OTHER, as_stream(stream));
-  launch(k_select, 1, kSelectThreads, dyn, as_stream(stream), d_score, d_pinned, N, a, d_group, d_order);
+  if (nc == 1)   // a lone CTA is a cluster of one: its cluster barriers and peer accesses stay in the CTA
+    launch(k_select, 1, kSelectThreads, dyn, as_stream(stream), d_score, d_pinned, N, a, d_group, d_order);
+  else
+    launch_cluster(k_select, nc, kSelectThreads, dyn, as_stream(stream), (unsigned)nc, d_score, d_pinned, N, a,
+                   d_group, d_order);
   count_launch(1);
   return check_launch("select launch");
 }
