@@ -277,40 +277,27 @@ def time_device(fn, steps, barrier):
 
 
 def time_e2e(step, x_host_np, n, barrier):
-    """ms for n iterations through the public API with host buffers: every iteration uploads its
-    latent from pinned host memory and downloads its result.  The latent is double-buffered on
-    the device, so iteration k+1's upload (H2D stream) and iteration k's download (D2H stream)
-    run while iteration k / k+1 computes; every copy is inside the timed region."""
+    """ms for n iterations through the C ABI's host-buffer entry point (hsa_iteration_host): every
+    iteration uploads its latent from pinned host memory, runs the full iteration (layer step on
+    every token, cached Euler with the fused score, regrouping) and downloads the updated latent.
+    Two device slots alternate, so the library overlaps iteration k+1's upload (H2D stream) and
+    iteration k's download (D2H stream) with compute; every copy is inside the timed region."""
     import torch
+    hsa = step.hsa
+    N, D = step.N, SHAPE.D
     hx = torch.from_numpy(x_host_np).pin_memory()
     hout = [torch.empty_like(hx).pin_memory() for _ in range(2)]
-    xs = [torch.empty(hx.shape, dtype=hx.dtype, device="cuda") for _ in range(2)]
+    slots = [hsa.HostSlot(N, D), hsa.HostSlot(N, D)]
     comp = torch.cuda.current_stream()
     h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
-    x_saved = step.x
+    m = step.model
 
     def run(count):
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_done = [torch.cuda.Event() for _ in range(2)]
-        with torch.cuda.stream(h2d):
-            xs[0].copy_(hx, non_blocking=True)
-            ev_in[0].record(h2d)
         for k in range(count):
-            b = k % 2
-            comp.wait_event(ev_in[b])
-            step.x = xs[b]
-            step.full()
-            ev_done[b].record(comp)
-            if k + 1 < count:
-                with torch.cuda.stream(h2d):
-                    if k >= 1:
-                        h2d.wait_event(ev_done[1 - b])     # iteration k-1 is done with that buffer
-                        h2d.wait_stream(d2h)               # ... and its result has been read back
-                    xs[1 - b].copy_(hx, non_blocking=True)
-                    ev_in[1 - b].record(h2d)
-            with torch.cuda.stream(d2h):
-                d2h.wait_event(ev_done[b])
-                hout[b].copy_(xs[b], non_blocking=True)
+            hsa.iteration_host(m.w, m.kc, m.vc, step.order, m.pos, m.xA, step.vhat, DSIGMA, hx, hout[k % 2],
+                               slots[k % 2], m.ws, ctx_k=m.ctx_k, ctx_v=m.ctx_v, score=step.score,
+                               group_sizes=step.sizes, group=step.group, order=step.order, sel_ws=step.sel_ws,
+                               stream=comp, stream_h2d=h2d, stream_d2h=d2h)
 
     run(2)                                                  # warm-up
     torch.cuda.synchronize()
@@ -324,7 +311,6 @@ def time_e2e(step, x_host_np, n, barrier):
     end.synchronize()
     torch.cuda.synchronize()
     barrier()
-    step.x = x_saved
     return start.elapsed_time(end)
 
 
@@ -400,7 +386,9 @@ def run_gpu(args, rank, world, barrier, allmax):
         e_ms = allmax(time_e2e(step, inp["x0"], n_e2e, barrier)) / n_e2e
         nbytes = GRID.N * SHAPE.D * 4
         e2e = {"value": round(e_ms, 4), "unit": "ms", "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
-               "overlap": "step k+1's upload and step k's download run on two copy streams during compute"}
+               "api": "hsa_iteration_host (C ABI, host buffers)",
+               "overlap": "two device slots: step k+1's upload and step k's download run on two copy streams "
+                          "during compute"}
 
     peak_sus, peak_burst, hbm, src = load_peaks()
     attn_per_step = attn_ms / args.steps

@@ -242,6 +242,61 @@ int hsa_layer_step(const hsa_layer_weights* w, void* d_kcache, void* d_vcache, i
                    const void* d_ctx_k, const void* d_ctx_v, int ctx_len, void* d_ws,
                    size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ one iteration, latent in host memory
+ * One HSA iteration (§2.1-§2.3) of a model made of one block, whose output rows are the velocity
+ * (C = D), for a caller that keeps the latent x in host memory between iterations.  The library
+ * moves it:
+ *   1. on stream_h2d: wait for slot->ev_free, copy h_x_in -> slot->d_x, record slot->ev_in;
+ *   2. on stream: wait for slot->ev_in; v_A = hsa_layer_step of the M active rows d_idx,
+ *      gathered from slot->d_x; hsa_euler_update (v_hat[A] = v_A, x += dsigma v_hat, and the L1
+ *      relative-change score into d_score when M == N and d_score is not NULL); when M == N and
+ *      d_group is not NULL, hsa_select_tokens regroups the tokens from that score into d_group
+ *      and d_order; record slot->ev_done;
+ *   3. on stream_d2h: wait for slot->ev_done, copy slot->d_x -> h_x_out, record slot->ev_free.
+ * h_x_in, h_x_out: host buffers of N x D float32 (page-locked, or the copies do not overlap
+ * compute); they may be the same buffer.  The device-side state (weights, caches, v_hat, the
+ * velocity rows d_xA, M x D, the scores and groups, the workspaces) is the caller's, as in
+ * hsa_layer_step, hsa_euler_update and hsa_select_tokens; d_order may be d_idx (a full step
+ * reads A_i before it regroups).  The events are cudaEvent_t handles (passed as void*) created by
+ * the caller, timing may be disabled; an event never recorded counts as complete.  A caller that
+ * alternates two slots overlaps the upload of iteration k + 1 and the download of iteration k
+ * with compute.  The three streams may be one stream (no overlap).  Copies are cudaMemcpyAsync.
+ * Returns the first failing status of the steps (nothing after it is enqueued). */
+typedef struct hsa_iteration_args {
+  const hsa_layer_weights* w;
+  void* d_kcache;               /* N x D, dtype of w                                         */
+  void* d_vcache;               /* N x D                                                     */
+  int N;
+  const int32_t* d_idx;         /* M active token indices (A_i)                              */
+  int M;
+  const int32_t* d_pos;         /* N x 3 (frame, row, column)                                */
+  const void* d_ctx_k;          /* ctx_len x D or NULL (no cross-attention)                   */
+  const void* d_ctx_v;
+  int ctx_len;
+  float* d_xA;                  /* M x D float32: the block's rows, v_A                      */
+  float* d_vhat;                /* N x D float32, updated                                    */
+  float dsigma;                 /* sigma_{i+1} - sigma_i                                     */
+  float* d_score;               /* N float32 or NULL                                         */
+  int K;                        /* groups of the regrouping                                  */
+  const int* h_group_sizes;     /* K sizes (host), sum N                                     */
+  int8_t* d_group;              /* N, or NULL: no regrouping                                 */
+  int32_t* d_order;             /* N                                                         */
+  void* d_ws;                   /* hsa_layer_step_workspace_size(M, D, F, dtype) bytes       */
+  size_t ws_bytes;
+  void* d_sel_ws;               /* hsa_select_tokens_workspace_size(N, K) bytes              */
+  size_t sel_ws_bytes;
+} hsa_iteration_args;
+
+typedef struct hsa_host_slot {
+  float* d_x;                   /* N x D float32 device copy of the latent                   */
+  void* ev_in;                  /* cudaEvent_t: upload done                                  */
+  void* ev_done;                /* cudaEvent_t: iteration done                               */
+  void* ev_free;                /* cudaEvent_t: download done, the slot may be refilled      */
+} hsa_host_slot;
+
+int hsa_iteration_host(const hsa_iteration_args* a, const float* h_x_in, float* h_x_out,
+                       const hsa_host_slot* slot, void* stream, void* stream_h2d, void* stream_d2h);
+
 /* ------------------------------------------------------------------ building blocks of the step
  * Full-context attention of §2.2 on its own: M compacted queries against L
  * cached keys/values, H heads of 128: o = softmax(q K^T / sqrt(128)) V.

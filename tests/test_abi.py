@@ -93,6 +93,28 @@ def test_device_calls_reject_bad_arguments_on_host(lib):
     assert b"need" in lib.hsa_last_error_string() or len(lib.hsa_last_error_string()) > 0
 
 
+def test_iteration_host_rejects_bad_arguments_on_host(lib):
+    """hsa_iteration_host checks every argument of its steps before it enqueues the upload."""
+    null = None
+    buf = (C.c_float * 4)()
+    slot = hsa.HostSlotC(None, None, None, None)
+    assert lib.hsa_iteration_host(null, buf, buf, C.byref(slot), null, null, null) == hsa.HSA_EINVAL
+    w = hsa.LayerWeightsC(256, 2, 1024, hsa.HSA_BF16)
+    a = hsa.IterationArgsC(C.pointer(w))
+    a.N, a.M = 8, 8
+    assert lib.hsa_iteration_host(C.byref(a), buf, buf, C.byref(slot), null, null, null) == hsa.HSA_EINVAL
+    assert b"events" in lib.hsa_last_error_string()
+    fake = 1 << 20                                         # 16-byte aligned stand-ins, never dereferenced
+    slot = hsa.HostSlotC(fake, fake, fake, fake)
+    assert lib.hsa_iteration_host(C.byref(a), buf, buf, C.byref(slot), null, null, null) == hsa.HSA_EINVAL
+    assert b"misaligned" in lib.hsa_last_error_string()    # the weights are NULL
+    a.M = 9                                                # M > N
+    assert lib.hsa_iteration_host(C.byref(a), buf, buf, C.byref(slot), null, null, null) == hsa.HSA_EINVAL
+    w.D = 300                                              # D != 128 H
+    a.M = 8
+    assert lib.hsa_iteration_host(C.byref(a), buf, buf, C.byref(slot), null, null, null) == hsa.HSA_EINVAL
+
+
 def test_workspace_sizes(lib):
     assert hsa.layer_step_workspace_size(32760, 1536, 8960, hsa.HSA_BF16) >= 32760 * (6 * 1536 + 8960) * 2
     assert hsa.layer_step_workspace_size(1024, 256, 1024, hsa.HSA_F32) >= 1024 * (6 * 256 + 1024) * 4

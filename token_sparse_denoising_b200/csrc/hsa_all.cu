@@ -8,5 +8,6 @@
 #include "attn_tc.cu"
 #include "simt_f32.cu"
 #include "api.cu"
+#include "host_io.cu"
 #include "shard.cu"
 #include "noalloc.cu"

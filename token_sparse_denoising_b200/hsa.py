@@ -36,6 +36,18 @@ class LayerWeightsC(C.Structure):
                 ("w_o2", vp), ("b_o2", vp)]
 
 
+class IterationArgsC(C.Structure):
+    _fields_ = [("w", C.POINTER(LayerWeightsC)), ("d_kcache", vp), ("d_vcache", vp), ("N", i32), ("d_idx", vp),
+                ("M", i32), ("d_pos", vp), ("d_ctx_k", vp), ("d_ctx_v", vp), ("ctx_len", i32), ("d_xA", vp),
+                ("d_vhat", vp), ("dsigma", f32), ("d_score", vp), ("K", i32), ("h_group_sizes", vp),
+                ("d_group", vp), ("d_order", vp), ("d_ws", vp), ("ws_bytes", sz), ("d_sel_ws", vp),
+                ("sel_ws_bytes", sz)]
+
+
+class HostSlotC(C.Structure):
+    _fields_ = [("d_x", vp), ("ev_in", vp), ("ev_done", vp), ("ev_free", vp)]
+
+
 _SIGS = {
     "hsa_last_error_string": (C.c_char_p, []),
     "hsa_device_status": (i32, [vp]),
@@ -69,6 +81,7 @@ _SIGS = {
     "hsa_qk_norm_rope_ext": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]),
     "hsa_rms_rows_ext": (i32, [vp, i32, i32, i32, i32, vp, i32, vp, i32, vp, vp]),
     "hsa_gated_residual": (i32, [vp, vp, i32, i32, vp, vp, vp]),
+    "hsa_iteration_host": (i32, [C.POINTER(IterationArgsC), vp, vp, C.POINTER(HostSlotC), vp, vp, vp]),
 }
 
 
@@ -344,6 +357,37 @@ def gated_residual(X, y, b=None, gate=None, stream=None):
     M, D = X.shape
     _check(lib().hsa_gated_residual(_ptr(X), _ptr(y), M, D, _ptr(b), _ptr(gate), _stream(stream)),
            "hsa_gated_residual")
+
+
+class HostSlot:
+    """A device copy of the latent (N x D float32) and the three events of one hsa_iteration_host
+    slot.  Each event is recorded once here, so that it exists and counts as complete."""
+
+    def __init__(self, N: int, D: int, device="cuda"):
+        import torch
+        self.x = torch.empty((N, D), dtype=torch.float32, device=device)
+        self.events = [torch.cuda.Event() for _ in range(3)]
+        for e in self.events:
+            e.record()
+        self.c = HostSlotC(_ptr(self.x), *(e.cuda_event for e in self.events))
+
+
+def iteration_host(w: "LayerWeights", kcache, vcache, idx, pos, xA, vhat, dsigma: float, h_x_in, h_x_out,
+                   slot: HostSlot, ws, ctx_k=None, ctx_v=None, score=None, group_sizes=None, group=None,
+                   order=None, sel_ws=None, stream=None, stream_h2d=None, stream_d2h=None):
+    """One iteration with the latent in host memory (hsa_iteration_host): h_x_in / h_x_out are CPU
+    tensors (N x D float32, pinned for overlap); the device state is as for layer_step,
+    euler_update and select_tokens."""
+    N, M = kcache.shape[0], idx.shape[0]
+    sizes = np.ascontiguousarray(group_sizes if group_sizes is not None else [N], np.int32)
+    a = IterationArgsC(C.pointer(w.c), _ptr(kcache), _ptr(vcache), N, _ptr(idx), M, _ptr(pos), _ptr(ctx_k),
+                       _ptr(ctx_v), 0 if ctx_k is None else ctx_k.shape[0], _ptr(xA), _ptr(vhat), dsigma,
+                       _ptr(score), len(sizes), sizes.ctypes.data, _ptr(group), _ptr(order), _ptr(ws),
+                       ws.numel() * ws.element_size(), _ptr(sel_ws),
+                       0 if sel_ws is None else sel_ws.numel() * sel_ws.element_size())
+    _check(lib().hsa_iteration_host(C.byref(a), h_x_in.data_ptr(), h_x_out.data_ptr(), C.byref(slot.c),
+                                    _stream(stream), _stream(stream_h2d), _stream(stream_d2h)),
+           "hsa_iteration_host")
 
 
 class LayerWeights:
