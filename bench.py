@@ -874,7 +874,7 @@ def measure_configs():
     """The other workloads, measured beside the headline step on the same GPU in the same run."""
     t0 = time.perf_counter()
     out = {"attention_euler_sweep": measure_sweep(),
-           "wan14_block": measure_wan14(patterns=("contiguous",), with_oracle=True),
+           "wan14_block": measure_wan14(with_oracle=True),
            "tiny_fp32_loop": measure_tiny(with_oracle=True), "wan13_loop": measure_loop(graph=False)}
     out["wall_s"] = round(time.perf_counter() - t0, 1)
     return out
