@@ -137,9 +137,15 @@ def _lin_case(seed, M, K, Nout, bf16):
 
 
 @pytest.mark.parametrize("M,K,Nout", [(300, 256, 768), (129, 128, 64), (1000, 512, 384), (1, 64, 128),
-                                      (4097, 1536, 512)])
+                                      (4097, 1536, 512),
+                                      # 256-column outputs with more than 128 rows: the two-CTA kernel;
+                                      # a pair whose second CTA holds one valid row, a single k-block,
+                                      # and a k-loop that wraps the six-stage ring several times
+                                      (129, 128, 256), (257, 64, 256), (2048, 1024, 2304)])
 @pytest.mark.parametrize("epi", [0, 1, 2, 3])
 def test_linear_bf16(cuda_lib, M, K, Nout, epi):
+    """bf16 linear layer against the oracle for every epilogue: outputs of 256 columns with more than
+    128 rows run the two-CTA (cta_group::2) kernel, the others the one-CTA kernel."""
     hsa = cuda_lib
     x, w, b, g, y0 = _lin_case(11, M, K, Nout, True)
     acc = O.linear(x, w, b)

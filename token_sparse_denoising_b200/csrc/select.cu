@@ -49,37 +49,6 @@ constexpr int kMaxGroups = 16;
 // a CTA with a longer range reads the scores from global memory on every pass.
 constexpr int kSelectStagedMax = 36864;
 
-// ---- cluster helpers: rank, distributed shared memory, barrier
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_size() {
-  uint32_t n;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
-  return n;
-}
-// address of the same shared-memory variable in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t peer_smem(const void* p, uint32_t rank) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
-  return a;
-}
-__device__ __forceinline__ uint32_t ld_peer(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_peer(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-// every thread of every CTA of the cluster; orders the shared-memory writes before it
-// (local and remote) before the reads after it
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 struct SelectArgs {
   int K;
   int staged;               // 1: each CTA's keys staged in dynamic shared memory
