@@ -183,7 +183,8 @@ def test_linear_f32(cuda_lib, M, K, Nout, epi):
                                           (257, 300, 3, 4.0), (130, 256, 2, 1.0), (100, 129, 1, 4.0),
                                           # more than 8 key tiles: the two-parity kernel
                                           (64, 4000, 2, 1.0), (130, 1100, 2, 1.0), (257, 1153, 3, 4.0),
-                                          (1, 1025, 1, 1.0), (128, 1152, 1, 1.0)])
+                                          (1, 1025, 1, 1.0), (128, 1152, 1, 1.0),
+                                          (256, 1153, 3, 4.0), (512, 3000, 2, 1.0), (250, 1500, 1, 1.0)])
 def test_attention_bf16(cuda_lib, M, L, H, qscale):
     """Key ranges of at most 8 tiles (1024 keys) run the one-parity kernel, longer ones the
     two-parity kernel: ragged query and key tiles of both, one query row, one key."""
