@@ -4,20 +4,26 @@
 //
 //   y[M x Nout] = epilogue(x[M x K] * W[Nout x K]^T + b)
 //
-// Persistent CTAs (one per SM) walk 128 x BN output tiles.  Warp roles:
-//   warp 0      TMA producer: A (128 x 64) and B (BN x 64) k-blocks into a ring
-//               of STAGES shared-memory slots, 128-byte swizzled;
-//   warp 1      allocates 2 x BN TMEM columns (two accumulators); the warp runs
-//               the loop converged and one elected lane issues tcgen05.mma
-//               (M=128, N=BN, K=16) into the free one and releases each
-//               shared-memory slot with tcgen05.commit;
-//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter, bias, GELU /
-//               residual gate.  Thread = output row.  Each warp stages 32 x 32
-//               sub-tiles of the output in shared memory and hands them to the TMA:
-//               bf16 and fp32 outputs by tensor stores, the fp32 residual update
-//               y += gate * (acc + b) by a tensor reduce-add done in L2, so the
-//               epilogue never waits on a global load.
-// Rows beyond M are zero-filled by TMA and never stored.
+// Two kernels share the epilogue (store_chunk):
+//   k_gemm_pair  outputs 256-column multiples with more than 128 rows (every GEMM of the block):
+//                a cluster of two CTAs on two SMs computes 256 x 256 tiles with one stream of
+//                tcgen05.mma.cta_group::2 issued by CTA 0; each CTA loads its own 128 rows of A and
+//                128 of the 256 weight rows per k-block, so each SM moves half the weight bytes per
+//                FLOP (details above the kernel);
+//   k_gemm_tc    everything else: one CTA per 128 x BN tile.
+// Both are persistent (one CTA, or pair, per SM walks the output tiles).  Warp roles:
+//   warp 0      TMA producer: A (128 x 64) and B (BN x 64, or 128 x 64 per CTA of a pair)
+//               k-blocks into a ring of shared-memory slots, 128-byte swizzled;
+//   warp 1      allocates the TMEM accumulators (two, so the epilogue of one tile overlaps the
+//               mainloop of the next); the warp runs the loop converged and one elected lane
+//               issues tcgen05.mma (M=128 or 256, N=BN, K=16) and releases each shared-memory
+//               slot with tcgen05.commit;
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quarter, bias, GELU / residual gate.
+//               Thread = output row.  Each warp stages 32 x 32 sub-tiles of the output in shared
+//               memory and hands them to the TMA: bf16 and fp32 outputs by tensor stores, the
+//               fp32 residual update y += gate * (acc + b) by a tensor reduce-add done in L2, so
+//               the epilogue never waits on a global load.
+// Rows beyond M are zero-filled by TMA and never stored.  No load is multicast.
 #include "tcgen05.cuh"
 
 namespace hsa {
