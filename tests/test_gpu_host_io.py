@@ -12,16 +12,16 @@ from token_sparse_denoising_b200 import pipeline, synthetic as S
 pytestmark = pytest.mark.gpu
 
 
-def _setup(hsa, seed):
+def _setup(hsa, seed, bf16=True):
     grid = S.Grid(2, 8, 10)
     N, D = grid.N, 256
     shape = S.BlockShape(D, 2, 512, True, 16)
-    bw = S.perturb_vectors(S.block_weights(seed, shape, True, 0.05), seed + 1)
+    bw = S.perturb_vectors(S.block_weights(seed, shape, bf16, 0.05), seed + 1)
     pos = S.token_positions(grid)
-    ctx = S.normal(seed + 4, (16, D), 1.0, True)
-    kc0, vc0 = S.normal(seed + 5, (N, D), 1.0, True), S.normal(seed + 6, (N, D), 1.0, True)
+    ctx = S.normal(seed + 4, (16, D), 1.0, bf16)
+    kc0, vc0 = S.normal(seed + 5, (N, D), 1.0, bf16), S.normal(seed + 6, (N, D), 1.0, bf16)
     x0, vh0 = S.normal(seed + 2, (N, D)), S.normal(seed + 3, (N, D))
-    model = pipeline.SingleBlockModel(bw, pos, N, bf16=True, ctx=ctx, cache_init=(kc0, vc0))
+    model = pipeline.SingleBlockModel(bw, pos, N, bf16=bf16, ctx=ctx, cache_init=(kc0, vc0))
     st = dict(model=model, x=torch.from_numpy(x0).cuda(), vhat=torch.from_numpy(vh0).cuda(),
               score=torch.zeros(N, device="cuda"), group=torch.zeros(N, dtype=torch.int8, device="cuda"),
               order=torch.arange(N, dtype=torch.int32, device="cuda"))
@@ -29,11 +29,13 @@ def _setup(hsa, seed):
     return st, x0
 
 
-@pytest.mark.parametrize("same_stream", [False, True])
-def test_iteration_host_matches_device_path(cuda_lib, same_stream):
+@pytest.mark.parametrize("same_stream,bf16", [(False, True), (True, True), (False, False)])
+def test_iteration_host_matches_device_path(cuda_lib, same_stream, bf16):
+    """bf16 (tensor-core kernels) and fp32 (CUDA-core kernels) blocks, with separate copy streams
+    and with everything on one stream."""
     hsa = cuda_lib
-    dev, x0 = _setup(hsa, 40)
-    hst, _ = _setup(hsa, 40)
+    dev, x0 = _setup(hsa, 40, bf16)
+    hst, _ = _setup(hsa, 40, bf16)
     N, D = x0.shape
     sizes = [N // 2, N - N // 2]
     # steps: full (regroup), the first group only, full, the first group only
