@@ -183,9 +183,9 @@ def test_binding_signatures_match_the_header():
         assert _ctype_kind(rtype) == want_ret, f"{name}: return {rtype} vs {ret}"
 
 
-def test_layer_weights_struct_matches_the_header():
+def _struct_fields(struct):
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
-    body = re.search(r"typedef struct hsa_layer_weights \{(.*?)\} hsa_layer_weights;", text, flags=re.S).group(1)
+    body = re.search(r"typedef struct %s \{(.*?)\} %s;" % (struct, struct), text, flags=re.S).group(1)
     fields = []
     for decl in body.split(";"):
         decl = decl.strip()
@@ -193,4 +193,30 @@ def test_layer_weights_struct_matches_the_header():
             continue
         names = decl.split(None, 1)[1] if not decl.startswith("const") else decl.split(None, 2)[2]
         fields += [n.strip().lstrip("*").strip() for n in names.split(",")]
-    assert fields == [f[0] for f in hsa.LayerWeightsC._fields_]
+    return fields
+
+
+@pytest.mark.parametrize("struct,cls", [("hsa_layer_weights", "LayerWeightsC"), ("hsa_iteration_args", "IterationArgsC"),
+                                        ("hsa_host_slot", "HostSlotC")])
+def test_struct_layouts_match_the_c_compiler(tmp_path, struct, cls):
+    """The ctypes mirrors of the header's structs have the same field names, order, offsets and size
+    as the C compiler gives them (gcc on this host, the same LP64 layout nvcc's host compiler uses)."""
+    import shutil
+    import subprocess
+    fields = _struct_fields(struct)
+    ctype = getattr(hsa, cls)
+    assert fields == [f[0] for f in ctype._fields_]
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "layout.c"
+    lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', 'int main(void) {',
+             f'  printf("%zu\\n", sizeof({struct}));']
+    lines += [f'  printf("%zu\\n", offsetof({struct}, {f}));' for f in fields]
+    lines += ['  return 0;', '}']
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-o", str(exe), str(src)], check=True, capture_output=True)
+    got = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    assert got[0] == C.sizeof(ctype)
+    assert got[1:] == [getattr(ctype, f).offset for f in fields]
