@@ -113,6 +113,23 @@ def test_iteration_host_rejects_bad_arguments_on_host(lib):
     w.D = 300                                              # D != 128 H
     a.M = 8
     assert lib.hsa_iteration_host(C.byref(a), buf, buf, C.byref(slot), null, null, null) == hsa.HSA_EINVAL
+    # every buffer present (aligned stand-ins): the regrouping arguments are checked too
+    w.D = 256
+    for name, _ in hsa.LayerWeightsC._fields_[4:15]:
+        setattr(w, name, fake)
+    for name in ("d_kcache", "d_vcache", "d_idx", "d_pos", "d_xA", "d_vhat", "d_ws", "d_score", "d_group",
+                 "d_order", "d_sel_ws"):
+        setattr(a, name, fake)
+    a.ws_bytes = lib.hsa_layer_step_workspace_size(8, 256, 1024, hsa.HSA_BF16) - 1
+    assert lib.hsa_iteration_host(C.byref(a), buf, buf, C.byref(slot), null, null, null) == hsa.HSA_EWORKSPACE
+    a.ws_bytes += 1
+    a.sel_ws_bytes = 1 << 20
+    sizes = (C.c_int * 2)(4, 5)                            # sums to 9, not N = 8
+    a.K, a.h_group_sizes = 2, C.cast(sizes, C.c_void_p)
+    assert lib.hsa_iteration_host(C.byref(a), buf, buf, C.byref(slot), null, null, null) == hsa.HSA_EINVAL
+    assert b"sum to N" in lib.hsa_last_error_string()
+    a.K = 17                                               # more groups than the selection supports
+    assert lib.hsa_iteration_host(C.byref(a), buf, buf, C.byref(slot), null, null, null) == hsa.HSA_EINVAL
 
 
 def test_workspace_sizes(lib):
