@@ -260,8 +260,11 @@ int hsa_layer_step(const hsa_layer_weights* w, void* d_kcache, void* d_vcache, i
  * reads A_i before it regroups).  The events are cudaEvent_t handles (passed as void*) created by
  * the caller, timing may be disabled; an event never recorded counts as complete.  A caller that
  * alternates two slots overlaps the upload of iteration k + 1 and the download of iteration k
- * with compute.  The three streams may be one stream (no overlap).  Copies are cudaMemcpyAsync.
- * Returns the first failing status of the steps (nothing after it is enqueued). */
+ * with compute.  The three streams may be one stream (no overlap).  Copies are cudaMemcpyAsync,
+ * and the call does not wait on the host: a caller that passes one call's h_x_out as a later
+ * call's h_x_in waits for the first call's ev_free first (cudaEventSynchronize).  Every argument
+ * is checked before anything is enqueued; a CUDA error after that returns HSA_ECUDA with the steps
+ * before it enqueued. */
 typedef struct hsa_iteration_args {
   const hsa_layer_weights* w;
   void* d_kcache;               /* N x D, dtype of w                                         */
